@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Throughput of the Muon / MuonGS optimizer step on B200.
+
+One step = one pass of the whole step (momentum, normalisation, 5 Newton-Schulz
+iterations, scale, projection / decay, update) over every matrix of a shape set,
+with weights, momenta and gradients resident in HBM. Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt160m]
+  python bench.py --impl reference ...   # the float64 CPU oracle on host cores
+
+Multi-GPU (torchrun, one process per GPU): the matrices of a shape set are
+independent, so each rank steps its own copy of the shape set with no collective
+on the data path (weak scaling); `value` counts the shape-set steps of all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="gpt160m")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), util=float(parts[4]),
+                                     reasons=[n for n, v in zip(
+                                         ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                                          "sw_power_cap"], parts[5:]) if v.lower() == "active"]))
+                except ValueError:
+                    continue
+        os.unlink(self.tmp.name)
+        load = [r for r in rows if r["util"] > 0] or rows
+        if not load:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({x for r in load for x in r["reasons"]})
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in load), "reasons": reasons,
+                "samples": len(load)}
+
+
+def gpu_id_for(torch, dev: int) -> str:
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+# ------------------------------------------------------------------ roofline traffic record
+def traffic_record(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, valid only
+    while the kernel's source is unchanged (sha256 of the sources listed there)."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        parts = dict(p.split("=", 1) for p in line.split() if "=" in p)
+        if parts.get("kernel") != kernel or parts.get("workload") != workload:
+            continue
+        h = hashlib.sha256()
+        for src in parts.get("sources", "").split(","):
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != parts.get("sha"):
+            return None
+        return float(parts["bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(w, run, budget_s: float, rotate: int = 0):
+    """Times the float64 oracle on a stratified sample of the shape set and extrapolates
+    to one full step: sum over shape classes of count x mean seconds per matrix."""
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+    from oracle import muon_oracle as orc
+    hp = orc.HParams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
+                     equilibrate=run.equilibrate)
+    specs = w.matrices()
+    by_class = {}
+    for s in specs:
+        by_class.setdefault((s.rows, s.cols), []).append(s)
+    t_start = time.perf_counter()
+    per_class, sampled = {}, 0
+    rounds = 0
+    while True:
+        for key, lst in by_class.items():
+            s = lst[(rotate + rounds) % len(lst)]
+            W = wl.weight(w, s).astype("float64")
+            G = wl.grad(w, s, 0).astype("float64")
+            M = __import__("numpy").zeros_like(W)
+            t0 = time.perf_counter()
+            orc.muon_step(W, G, M, hp)
+            per_class.setdefault(key, []).append(time.perf_counter() - t0)
+            sampled += 1
+        rounds += 1
+        if time.perf_counter() - t_start >= budget_s or rounds >= 64:
+            break
+    est = sum(len(by_class[k]) * statistics.mean(v) for k, v in per_class.items())
+    return est, sampled, rounds
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    run = w.runs[0]
+    per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    for i in range(args.warmup):
+        oracle_sample(w, run, 0.0, rotate=i)
+    times, sampled = [], 0
+    for i in range(args.steps):
+        est, n, _ = oracle_sample(w, run, per_step, rotate=args.warmup + i)
+        times.append(est)
+        sampled += n
+    mean_s = statistics.mean(times)
+    value = 1.0 / mean_s
+    cores = blas_threads()
+    sample = (f"each step: float64 oracle on a stratified sample of the {w.name} shape set "
+              f"(>= 1 matrix per shape class, about {per_step:.0f} s), extrapolated by class counts; "
+              f"{sampled} matrices timed in total")
+    line = {"metric": "muon_steps_per_s", "value": value, "unit": "steps/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "matrices": w.n_matrices, "params": w.n_params,
+                       "mode": run.mode, "weight_decay": run.weight_decay,
+                       "equilibrate": run.equilibrate},
+            "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from matrix_orthogonalising_optimizer_03_b200 import binding as B
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    B.load()
+    w = wl.WORKLOADS[args.workload]
+    run = w.runs[0]
+    specs = w.matrices()
+    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    gsz = 2 if w.grad_dtype == "bf16" else 4
+
+    # resident inputs: W (fp32), M (fp32, zero), G (one flat buffer, views per matrix)
+    numel = sum(s.rows * s.cols for s in specs)
+    g_flat = torch.empty(numel, dtype=gdt, device=dev)
+    g_host = torch.empty(numel, dtype=gdt, pin_memory=True)
+    Ws, Ms, Gs = [], [], []
+    off = 0
+    for s in specs:
+        Ws.append(torch.from_numpy(wl.weight(w, s)).to(dev))
+        Ms.append(torch.zeros(s.rows, s.cols, dtype=torch.float32, device=dev))
+        gv = g_host[off:off + s.rows * s.cols].view(s.rows, s.cols)
+        gv.copy_(torch.from_numpy(wl.grad(w, s, 0)).to(gdt))
+        Gs.append(g_flat[off:off + s.rows * s.cols].view(s.rows, s.cols))
+        off += s.rows * s.cols
+    g_flat.copy_(g_host)
+    hp = B.hparams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
+                   equilibrate=run.equilibrate, ns_fp32=w.ns_fp32)
+    plan = B.Plan(Ws, Gs, Ms, hp)
+    stats = B.new_stats(len(specs), dev)
+    stats_host = torch.empty_like(stats, device="cpu").pin_memory()
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(gpu_id_for(torch, local))
+    for _ in range(args.warmup):
+        plan.step(stats=stats)
+    torch.cuda.synchronize()
+    if plan.query_device_status() != 0:
+        raise RuntimeError("device-side error during warm-up")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # 1) device-timed region: K steps, inputs resident (W+M+G far larger than L2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        plan.step(stats=stats)
+    e1.record(stream)
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    clocks = sampler.stop()
+
+    # 2) profiled pass (same K steps): per-kernel device times on the launching stream
+    B.load().muon_plan_profile_enable(plan._plan, 1)
+    barrier()
+    for _ in range(args.steps):
+        plan.step(stats=stats)
+    prof = plan_profile(B, plan)
+    B.load().muon_plan_profile_enable(plan._plan, 0)
+    launches_per_step = sum(p["launches"] for p in prof.values()) / args.steps
+
+    # 3) end to end through the public API: pinned H2D of the step's gradients,
+    #    the step, and a D2H read of the per-matrix statistics, every step
+    barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        g_flat.copy_(g_host, non_blocking=True)
+        plan.step(stats=stats)
+        stats_host.copy_(stats, non_blocking=True)
+    f1.record(stream)
+    barrier()
+    ms_e2e = max_over_ranks(f0.elapsed_time(f1))
+    if plan.query_device_status() != 0:
+        raise RuntimeError("device-side error in the timed region")
+
+    peaks, peak_src = load_peaks()
+    roof = roofline(prof, w, peaks, peak_src, args.workload)
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        est, n, rounds = oracle_sample(w, run, args.cpu_seconds)
+        cpu = {"value": 1.0 / est, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"float64 oracle on {n} matrices ({rounds} per shape class) of the "
+                         f"{w.name} shape set, extrapolated to one full step by class counts"}
+    if rank == 0:
+        steps_all = args.steps * world
+        line = {
+            "metric": "muon_steps_per_s", "value": steps_all / (ms / 1e3), "unit": "steps/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32" if w.ns_fp32 else "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "matrices": w.n_matrices, "params": w.n_params,
+                       "mode": run.mode, "weight_decay": run.weight_decay,
+                       "equilibrate": run.equilibrate, "ns_steps": 5, "grad_dtype": w.grad_dtype,
+                       "ns_tflops_per_step": wl.workload_ns_flops(w) / 1e12,
+                       "l2": "inputs larger than L2 (W+M+G = %.0f MB vs 126 MB)" % (
+                           numel * (8 + gsz) / 1e6),
+                       "parallelism": f"replica x{world}"},
+            "ns_tflops": wl.workload_ns_flops(w) * args.steps / (ms / 1e3) / 1e12,
+            "roofline": roof,
+            "kernels": {k: {"launches_per_step": v["launches"] / args.steps,
+                            "ms_per_step": v["total_ms"] / args.steps} for k, v in prof.items()
+                        if v["launches"]},
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "e2e": {"value": steps_all / (ms_e2e / 1e3), "unit": "steps/s",
+                    "h2d_bytes_per_step": numel * gsz, "d2h_bytes_per_step": stats.numel() * 4},
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    plan.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def plan_profile(B, plan):
+    import ctypes
+
+    class Entry(ctypes.Structure):
+        _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32),
+                    ("total_ms", ctypes.c_float), ("flops", ctypes.c_double),
+                    ("bytes", ctypes.c_double)]
+    lib = B.load()
+    lib.muon_plan_profile_read.restype = ctypes.c_int
+    lib.muon_plan_profile_read.argtypes = [ctypes.c_void_p, ctypes.POINTER(Entry), ctypes.c_int]
+    arr = (Entry * 16)()
+    n = lib.muon_plan_profile_read(plan._plan, arr, 16)
+    if n < 0:
+        raise RuntimeError("muon_plan_profile_read failed")
+    return {arr[i].name.decode(): {"launches": arr[i].launches, "total_ms": arr[i].total_ms,
+                                    "flops": arr[i].flops, "bytes": arr[i].bytes} for i in range(n)}
+
+
+def roofline(prof, w, peaks, peak_src, workload):
+    ns = {k: v for k, v in prof.items() if k.startswith("ns_") and v["launches"]}
+    if not ns:
+        return None
+    name, v = max(ns.items(), key=lambda kv: kv[1]["total_ms"])
+    per_launch_s = v["total_ms"] / 1e3 / v["launches"]
+    flops = v["flops"] / v["launches"]
+    achieved = flops / per_launch_s / 1e12
+    if w.ns_fp32:
+        return {"bound": "alu", "kernel": name, "achieved": achieved, "unit": "TFLOP/s",
+                "peak": 148 * 128 * 2 * 1.965e9 / 1e12, "frac": None, "traffic": None,
+                "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x 1965 MHz"}
+    peak = peaks["bf16_tflops"]
+    traffic = traffic_record(name, workload)
+    return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+            "flops_per_launch": flops, "launch_ms": per_launch_s * 1e3,
+            "peak_source": f"{peak_src} bf16 (burst)"}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,281 @@
+"""ctypes binding of libmuon.so (C ABI in include/muon.h).
+
+Argument marshalling only: every step of the Muon update runs in the library's
+CUDA kernels. PyTorch supplies device memory and streams. The functions here
+raise `MuonError` when the library is missing or a call fails; there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_float, c_int, c_int32, c_int64, c_size_t, c_uint32, c_void_p
+from typing import List, Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmuon.so")
+
+MUON_OK = 0
+STATUS_NAMES = {
+    0: "MUON_OK", 1: "MUON_ERR_INVALID_ARG", 2: "MUON_ERR_SHAPE", 3: "MUON_ERR_DTYPE",
+    4: "MUON_ERR_ALIAS", 5: "MUON_ERR_WORKSPACE", 6: "MUON_ERR_CUDA", 7: "MUON_ERR_TIMEOUT",
+    8: "MUON_ERR_UNSUPPORTED",
+}
+MUON_F32, MUON_BF16 = 0, 1
+MUON_MODE_MUON, MUON_MODE_MUONGS = 0, 1
+MUON_SCALE_MOONLIGHT, MUON_SCALE_KELLER, MUON_SCALE_NONE = 0, 1, 2
+MUON_NESTEROV, MUON_EQUILIBRATE, MUON_NS_FP32, MUON_WANT_STATS = 1, 2, 4, 8
+
+MODES = {"muon": MUON_MODE_MUON, "muongs": MUON_MODE_MUONGS}
+SCALES = {"moonlight": MUON_SCALE_MOONLIGHT, "keller": MUON_SCALE_KELLER, "none": MUON_SCALE_NONE}
+
+
+class MuonError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}" if what else
+                         STATUS_NAMES.get(status, str(status)))
+
+
+class MuonMatrix(ctypes.Structure):
+    _fields_ = [("W", c_void_p), ("grad", c_void_p), ("momentum", c_void_p),
+                ("rows", c_int64), ("cols", c_int64),
+                ("ld_w", c_int64), ("ld_g", c_int64), ("ld_m", c_int64),
+                ("w_dtype", c_int32), ("g_dtype", c_int32)]
+
+
+class MuonHParams(ctypes.Structure):
+    _fields_ = [("lr", c_float), ("momentum", c_float), ("weight_decay", c_float),
+                ("ns_coeffs", c_float * 3), ("ns_steps", c_int32), ("eps", c_float),
+                ("mode", c_int32), ("scale", c_int32), ("scale_k", c_float), ("flags", c_uint32)]
+
+
+class MuonStats(ctypes.Structure):
+    _fields_ = [("w_norm", c_float), ("w_dot_o", c_float), ("o_norm", c_float),
+                ("update_rms", c_float), ("equil_axis", c_int32), ("reserved", c_int32)]
+
+
+class MuonNSMatrix(ctypes.Structure):
+    _fields_ = [("X", c_void_p), ("O", c_void_p), ("rows", c_int64), ("cols", c_int64),
+                ("ld_x", c_int64), ("ld_o", c_int64), ("dtype", c_int32), ("reserved", c_int32)]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Loads libmuon.so and declares its signatures. Raises if the library is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise MuonError(-1, f"libmuon.so not found at {path}; build it with "
+                            "`python -m matrix_orthogonalising_optimizer_03_b200.build`")
+    lib = ctypes.CDLL(path)
+    P = POINTER
+    sig = {
+        "muon_abi_version": (c_int, []),
+        "muon_status_string": (ctypes.c_char_p, [c_int]),
+        "muon_hparams_default": (c_int, [P(MuonHParams)]),
+        "muon_validate": (c_int, [P(MuonMatrix), c_int, P(MuonHParams)]),
+        "muon_workspace_size": (c_size_t, [P(MuonMatrix), c_int, P(MuonHParams)]),
+        "muon_step_batched": (c_int, [P(MuonMatrix), c_int, P(MuonHParams), c_void_p, c_size_t,
+                                      c_void_p, c_void_p]),
+        "muon_plan_create": (c_int, [P(MuonMatrix), c_int, P(MuonHParams), P(c_void_p)]),
+        "muon_plan_workspace_size": (c_size_t, [c_void_p]),
+        "muon_plan_set_hparams": (c_int, [c_void_p, P(MuonHParams)]),
+        "muon_plan_step": (c_int, [c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+        "muon_plan_destroy": (None, [c_void_p]),
+        "muon_ns_workspace_size": (c_size_t, [P(MuonNSMatrix), c_int, P(MuonHParams)]),
+        "muon_newton_schulz_batched": (c_int, [P(MuonNSMatrix), c_int, P(MuonHParams), c_void_p,
+                                               c_size_t, c_void_p]),
+        "muon_query_device_status": (c_int, [c_void_p, c_void_p]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    if lib.muon_abi_version() != 1:
+        raise MuonError(-1, "unexpected libmuon ABI version")
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != MUON_OK:
+        raise MuonError(status, what)
+
+
+def hparams(lr: float = 0.02, momentum: float = 0.95, weight_decay: float = 0.0,
+            ns_coeffs: Sequence[float] = (3.4445, -4.7750, 2.0315), ns_steps: int = 5,
+            eps: float = 1e-7, mode: str = "muon", scale: str = "moonlight", scale_k: float = 0.2,
+            nesterov: bool = True, equilibrate: bool = False, ns_fp32: bool = False) -> MuonHParams:
+    hp = MuonHParams()
+    _check(load().muon_hparams_default(ctypes.byref(hp)), "muon_hparams_default")
+    hp.lr, hp.momentum, hp.weight_decay = lr, momentum, weight_decay
+    hp.ns_coeffs[0], hp.ns_coeffs[1], hp.ns_coeffs[2] = ns_coeffs
+    hp.ns_steps, hp.eps = ns_steps, eps
+    hp.mode, hp.scale, hp.scale_k = MODES[mode], SCALES[scale], scale_k
+    hp.flags = ((MUON_NESTEROV if nesterov else 0) | (MUON_EQUILIBRATE if equilibrate else 0) |
+                (MUON_NS_FP32 if ns_fp32 else 0))
+    return hp
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return MUON_F32
+    if t.dtype == torch.bfloat16:
+        return MUON_BF16
+    raise MuonError(3, f"unsupported dtype {t.dtype}")
+
+
+def _check_2d(t, name: str):
+    if t.dim() != 2:
+        raise MuonError(2, f"{name} must be 2-D (got {t.dim()}-D)")
+    if t.stride(1) != 1 and t.size(1) > 1:
+        raise MuonError(2, f"{name} must be row-major with unit column stride")
+    if not t.is_cuda:
+        raise MuonError(1, f"{name} must be a CUDA tensor")
+
+
+def matrix_array(params, grads, momenta):
+    """The muon_matrix_t array for lists of W (fp32), G (fp32/bf16), M (fp32) tensors."""
+    n = len(params)
+    if len(grads) != n or len(momenta) != n:
+        raise MuonError(1, "params, grads and momenta must have the same length")
+    arr = (MuonMatrix * n)()
+    for i, (w, g, m) in enumerate(zip(params, grads, momenta)):
+        for t, nm in ((w, "W"), (g, "grad"), (m, "momentum")):
+            _check_2d(t, nm)
+        if tuple(g.shape) != tuple(w.shape) or tuple(m.shape) != tuple(w.shape):
+            raise MuonError(2, "W, grad and momentum shapes differ")
+        arr[i] = MuonMatrix(w.data_ptr(), g.data_ptr(), m.data_ptr(), w.size(0), w.size(1),
+                            max(w.stride(0), w.size(1)), max(g.stride(0), g.size(1)),
+                            max(m.stride(0), m.size(1)), _dtype_code(w), _dtype_code(g))
+    return arr
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _stats_ptr(stats) -> Optional[int]:
+    if stats is None:
+        return None
+    torch = _torch()
+    if stats.dtype != torch.int32 or stats.numel() % 6 != 0 or not stats.is_cuda:
+        raise MuonError(1, "stats must be a CUDA int32 tensor of n*6 elements")
+    return stats.data_ptr()
+
+
+def new_stats(n: int, device="cuda"):
+    """A device buffer for n muon_stats_t (int32 storage; see `decode_stats`)."""
+    return _torch().zeros((n, 6), dtype=_torch().int32, device=device)
+
+
+def decode_stats(stats) -> List[dict]:
+    torch = _torch()
+    s = stats.detach().cpu()
+    f = s.view(torch.float32)
+    return [dict(w_norm=float(f[i, 0]), w_dot_o=float(f[i, 1]), o_norm=float(f[i, 2]),
+                 update_rms=float(f[i, 3]), equil_axis=int(s[i, 4])) for i in range(s.shape[0])]
+
+
+def new_workspace(nbytes: int, device="cuda"):
+    """A 256-byte aligned device workspace (torch allocations are 512-byte aligned)."""
+    ws = _torch().empty(max(int(nbytes), 1), dtype=_torch().uint8, device=device)
+    if ws.data_ptr() % 256:
+        raise MuonError(5, "workspace allocation is not 256-byte aligned")
+    return ws
+
+
+def workspace_size(params, grads, momenta, hp: MuonHParams) -> int:
+    arr = matrix_array(params, grads, momenta)
+    return int(load().muon_workspace_size(arr, len(arr), ctypes.byref(hp)))
+
+
+def step_batched(params, grads, momenta, hp: MuonHParams, workspace=None, stats=None,
+                 stream=None):
+    """One Muon step over the lists (muon_step_batched). Returns the workspace used."""
+    lib = load()
+    arr = matrix_array(params, grads, momenta)
+    n = len(arr)
+    if workspace is None:
+        size = lib.muon_workspace_size(arr, n, ctypes.byref(hp))
+        if n and size == 0:
+            _check(lib.muon_validate(arr, n, ctypes.byref(hp)), "muon_validate")
+        workspace = new_workspace(size, params[0].device if n else "cuda")
+    _check(lib.muon_step_batched(arr, n, ctypes.byref(hp), workspace.data_ptr(), workspace.numel(),
+                                 _stats_ptr(stats), _stream_ptr(stream)), "muon_step_batched")
+    return workspace
+
+
+class Plan:
+    """A cached plan (muon_plan_*) over a fixed list of matrices, owning its workspace."""
+
+    def __init__(self, params, grads, momenta, hp: MuonHParams, workspace=None):
+        self._lib = load()
+        self._arr = matrix_array(params, grads, momenta)
+        self._keep = (list(params), list(grads), list(momenta))
+        self.n = len(self._arr)
+        self.hp = hp
+        h = c_void_p()
+        _check(self._lib.muon_plan_create(self._arr, self.n, ctypes.byref(hp), ctypes.byref(h)),
+               "muon_plan_create")
+        self._plan = h
+        self.workspace_bytes = int(self._lib.muon_plan_workspace_size(h))
+        dev = params[0].device if self.n else "cuda"
+        self.workspace = workspace if workspace is not None else new_workspace(self.workspace_bytes, dev)
+
+    def set_hparams(self, hp: MuonHParams):
+        _check(self._lib.muon_plan_set_hparams(self._plan, ctypes.byref(hp)), "muon_plan_set_hparams")
+        self.hp = hp
+
+    def step(self, stats=None, stream=None):
+        _check(self._lib.muon_plan_step(self._plan, self.workspace.data_ptr(), self.workspace.numel(),
+                                        _stats_ptr(stats), _stream_ptr(stream)), "muon_plan_step")
+
+    def query_device_status(self, stream=None) -> int:
+        return int(self._lib.muon_query_device_status(self.workspace.data_ptr(), _stream_ptr(stream)))
+
+    def close(self):
+        if getattr(self, "_plan", None):
+            self._lib.muon_plan_destroy(self._plan)
+            self._plan = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def newton_schulz(xs, outs, hp: MuonHParams, workspace=None, stream=None):
+    """O_i = NS(X_i / (||X_i||_F + eps)) for lists of 2-D CUDA tensors (fp32 or bf16)."""
+    lib = load()
+    n = len(xs)
+    arr = (MuonNSMatrix * n)()
+    for i, (x, o) in enumerate(zip(xs, outs)):
+        _check_2d(x, "X")
+        _check_2d(o, "O")
+        if x.dtype != o.dtype or tuple(x.shape) != tuple(o.shape):
+            raise MuonError(3, "X and O must have the same dtype and shape")
+        arr[i] = MuonNSMatrix(x.data_ptr(), o.data_ptr(), x.size(0), x.size(1),
+                              max(x.stride(0), x.size(1)), max(o.stride(0), o.size(1)),
+                              _dtype_code(x), 0)
+    if workspace is None:
+        size = lib.muon_ns_workspace_size(arr, n, ctypes.byref(hp))
+        workspace = new_workspace(size, xs[0].device if n else "cuda")
+    _check(lib.muon_newton_schulz_batched(arr, n, ctypes.byref(hp), workspace.data_ptr(),
+                                          workspace.numel(), _stream_ptr(stream)),
+           "muon_newton_schulz_batched")
+    return workspace

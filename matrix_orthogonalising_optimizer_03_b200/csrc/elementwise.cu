@@ -1,0 +1,449 @@
+// Memory-bound kernels of the Muon step (CUDA cores, HBM bound).
+//
+//   ingest        a1 momentum M = mu*M + G, a2 Nesterov U = G + mu*M, ||U||_F^2,
+//                 and U written to the Newton-Schulz slab in the oriented frame
+//                 (transposed through shared memory for tall matrices).
+//   post_reduce   ||W||^2, <W,O>, ||O||^2 and, for equilibration, per-row and
+//                 per-column sums of O^2 and W*O (storage frame).
+//   post_finalize one block per matrix: equilibration axis and factors (a6),
+//                 scale (a7), GS coefficient (a8), statistics, update coefficients.
+//   post_apply    a9: W <- cw*W + co*D*O (or, Newton-Schulz only, O out).
+//
+// Work unit: a 32 x 64 tile of the matrix in its storage frame, 256 threads,
+// 8 consecutive columns per thread (128-bit accesses when aligned). The tile
+// of each block is found by binary search over a per-matrix tile prefix.
+#include <cuda_runtime.h>
+
+#include "muon_internal.h"
+#include "ptx.cuh"
+
+namespace muon {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kTR = kElemTileR;  // 32 rows
+constexpr int kTC = kElemTileC;  // 64 cols
+
+__device__ __forceinline__ void load8_f32(const float* p, bool vec, int valid, float (&v)[8]) {
+  if (vec && valid == 8) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 y = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = e < valid ? p[e] : 0.f;
+  }
+}
+__device__ __forceinline__ void store8_f32(float* p, bool vec, int valid, const float (&v)[8]) {
+  if (vec && valid == 8) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (e < valid) p[e] = v[e];
+  }
+}
+__device__ __forceinline__ void load8_bf16(const uint16_t* p, bool vec, int valid, float (&v)[8]) {
+  if (vec && valid == 8) {
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = __uint_as_float(w[e] << 16);
+      v[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = e < valid ? bf16_to_f32(p[e]) : 0.f;
+  }
+}
+__device__ __forceinline__ void store8_bf16(uint16_t* p, bool vec, int valid, const float (&v)[8]) {
+  if (vec && valid == 8) {
+    uint4 x;
+    x.x = pack_bf16x2(v[0], v[1]);
+    x.y = pack_bf16x2(v[2], v[3]);
+    x.z = pack_bf16x2(v[4], v[5]);
+    x.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = x;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (e < valid) p[e] = f32_to_bf16(v[e]);
+  }
+}
+
+// Reads 8 values of the slab entry (oriented frame) at (row, col..col+7).
+__device__ __forceinline__ void load8_slab(const void* base, int x_fp32, int64_t off, int valid,
+                                           float (&v)[8]) {
+  if (x_fp32) load8_f32(static_cast<const float*>(base) + off, true, valid, v);
+  else load8_bf16(static_cast<const uint16_t*>(base) + off, true, valid, v);
+}
+__device__ __forceinline__ void store8_slab(void* base, int x_fp32, int64_t off, int valid,
+                                            const float (&v)[8]) {
+  if (x_fp32) store8_f32(static_cast<float*>(base) + off, true, valid, v);
+  else store8_bf16(static_cast<uint16_t*>(base) + off, true, valid, v);
+}
+
+template <int NV>
+__device__ __forceinline__ void block_sum(double (&v)[NV], double (*sh)[kThreads / 32]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    v[i] = warp_sum(v[i]);
+    if (lane == 0) sh[i][warp] = v[i];
+  }
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      double x = lane < kThreads / 32 ? sh[i][lane] : 0.0;
+      v[i] = warp_sum(x);
+    }
+  }
+}
+
+// Loads, for this thread's 8 storage-frame elements, the Newton-Schulz result O.
+// Tall matrices hold O^T in the slab: the block stages a 64 x 32 slab tile in
+// shared memory and reads it transposed. Block-uniform control flow.
+__device__ __forceinline__ void load_o_tile(const ElemArgs& a, const DevMat& d, const DevSlab& s,
+                                            int r0, int c0, float (*tile)[kTR + 1],
+                                            float (&o)[8]) {
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const int r = r0 + lr, c = c0 + lc;
+  if (!(d.flags & MAT_TRANSPOSED)) {
+    const int valid = (r < d.rows) ? min(8, d.cols - c) : 0;
+    if (valid > 0) load8_slab(s.xf, a.x_fp32, (int64_t)r * s.ldx + c, valid, o);
+    else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) o[e] = 0.f;
+    }
+  } else {
+    // slab rows = storage columns c0..c0+63, slab columns = storage rows r0..r0+31
+    const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
+    float v[8];
+    const int valid = (sr < d.cols) ? min(8, d.rows - sc) : 0;
+    if (valid > 0) load8_slab(s.xf, a.x_fp32, (int64_t)sr * s.ldx + sc, valid, v);
+    else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tile[threadIdx.x >> 2][(threadIdx.x & 3) * 8 + e] = v[e];
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = tile[lc + e][lr];
+  }
+}
+
+__device__ __forceinline__ int find_matrix(const ElemArgs& a, int b) {
+  int lo = 0, hi = a.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(a.tile_prefix + mid) <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// ------------------------------------------------------------------ ingest
+__global__ void __launch_bounds__(kThreads) ingest_kernel(const ElemArgs a) {
+  __shared__ float tile[kTC][kTR + 1];
+  __shared__ double red[1][kThreads / 32];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int tiles_c = (d.cols + kTC - 1) / kTC;
+  const int r0 = (t / tiles_c) * kTR, c0 = (t % tiles_c) * kTC;
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const int r = r0 + lr, c = c0 + lc;
+  const bool vec = (d.flags & MAT_VEC_OK) != 0;
+  const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+
+  float u[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) u[e] = 0.f;
+  if (valid > 0) {
+    float g[8];
+    if (d.flags & MAT_G_BF16)
+      load8_bf16(static_cast<const uint16_t*>(d.G) + (int64_t)r * d.ld_g + c, vec, valid, g);
+    else
+      load8_f32(static_cast<const float*>(d.G) + (int64_t)r * d.ld_g + c, vec, valid, g);
+    if (a.ns_only) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) u[e] = g[e];
+    } else {
+      float m[8];
+      float* mp = d.M + (int64_t)r * d.ld_m + c;
+      load8_f32(mp, vec, valid, m);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        m[e] = fmaf(a.mu, m[e], g[e]);                  // M_t = mu*M_{t-1} + G_t
+        u[e] = a.nesterov ? fmaf(a.mu, m[e], g[e]) : m[e];  // U = G_t + mu*M_t
+      }
+      store8_f32(mp, vec, valid, m);
+    }
+  }
+  double acc[1] = {0.0};
+  {
+    float sq = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      // the slab holds U rounded to its storage type; ||U|| is taken of that value
+      const float q = a.x_fp32 ? u[e] : bf16_to_f32(f32_to_bf16(u[e]));
+      sq = fmaf(q, q, sq);
+    }
+    acc[0] = sq;
+  }
+
+  if (!(d.flags & MAT_TRANSPOSED)) {
+    if (valid > 0) store8_slab(s.x0, a.x_fp32, (int64_t)r * s.ldx + c, valid, u);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tile[lc + e][lr] = u[e];
+    __syncthreads();
+    const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
+    const int v2 = (sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
+    if (v2 > 0) {
+      float w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = tile[threadIdx.x >> 2][(threadIdx.x & 3) * 8 + e];
+      store8_slab(s.x0, a.x_fp32, (int64_t)sr * s.ldx + sc, v2, w);
+    }
+  }
+  block_sum<1>(acc, red);
+  if (threadIdx.x == 0) atomicAdd(&a.scal[k].u2, acc[0]);
+}
+
+__device__ __forceinline__ float slab_scale(const ElemArgs& a, int k) {
+  if (!a.xs_from_u2) return 1.f;
+  return static_cast<float>(1.0 / (sqrt(a.scal[k].u2) + (double)a.eps));
+}
+
+// ------------------------------------------------------------------ post_reduce
+__global__ void __launch_bounds__(kThreads) post_reduce_kernel(const ElemArgs a) {
+  __shared__ float tile[kTC][kTR + 1];
+  __shared__ double red[3][kThreads / 32];
+  __shared__ float col_o2[kTC], col_wo[kTC];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int tiles_c = (d.cols + kTC - 1) / kTC;
+  const int r0 = (t / tiles_c) * kTR, c0 = (t % tiles_c) * kTC;
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const int r = r0 + lr, c = c0 + lc;
+  const bool vec = (d.flags & MAT_VEC_OK) != 0;
+  const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+  if (a.equilibrate && threadIdx.x < kTC) {
+    col_o2[threadIdx.x] = 0.f;
+    col_wo[threadIdx.x] = 0.f;
+  }
+
+  float o[8];
+  load_o_tile(a, d, s, r0, c0, tile, o);
+  const float xs = slab_scale(a, k);
+  float w[8];
+  if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w);
+  else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w[e] = 0.f;
+  }
+  float ww = 0.f, wo = 0.f, oo = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    o[e] *= xs;
+    ww = fmaf(w[e], w[e], ww);
+    wo = fmaf(w[e], o[e], wo);
+    oo = fmaf(o[e], o[e], oo);
+  }
+  if (a.equilibrate) {
+    // per-row sums: the 8 threads of a row are consecutive lanes
+    float ro = oo, rw = wo;
+#pragma unroll
+    for (int m = 4; m > 0; m >>= 1) {
+      ro += __shfl_xor_sync(0xffffffffu, ro, m);
+      rw += __shfl_xor_sync(0xffffffffu, rw, m);
+    }
+    if ((threadIdx.x & 7) == 0 && r < d.rows) {
+      atomicAdd(a.eq_o2 + s.eq_off + r, ro);
+      atomicAdd(a.eq_wo + s.eq_off + r, rw);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (e < valid) {
+        atomicAdd(&col_o2[lc + e], o[e] * o[e]);
+        atomicAdd(&col_wo[lc + e], w[e] * o[e]);
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < kTC && c0 + (int)threadIdx.x < d.cols) {
+      atomicAdd(a.eq_o2 + s.eq_off + d.rows + c0 + threadIdx.x, col_o2[threadIdx.x]);
+      atomicAdd(a.eq_wo + s.eq_off + d.rows + c0 + threadIdx.x, col_wo[threadIdx.x]);
+    }
+  }
+  double acc[3] = {ww, wo, oo};
+  block_sum<3>(acc, red);
+  if (threadIdx.x == 0) {
+    atomicAdd(&a.scal[k].w2, acc[0]);
+    atomicAdd(&a.scal[k].wo, acc[1]);
+    atomicAdd(&a.scal[k].o2, acc[2]);
+  }
+}
+
+// ------------------------------------------------------------------ post_finalize
+__device__ __forceinline__ double block_sum2(double& x, double& y, double (*sh)[kThreads / 32]) {
+  double v[2] = {x, y};
+  block_sum<2>(v, sh);
+  __shared__ double out[2];
+  if (threadIdx.x == 0) { out[0] = v[0]; out[1] = v[1]; }
+  __syncthreads();
+  x = out[0];
+  y = out[1];
+  __syncthreads();
+  return x;
+}
+
+__global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs a) {
+  __shared__ double red[2][kThreads / 32];
+  const int k = blockIdx.x;
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const MatScalars sc = a.scal[k];
+  const double rows = d.rows, cols = d.cols;
+  double scale = 1.0;
+  if (a.scale_rule == MUON_SCALE_MOONLIGHT) scale = (double)a.scale_k * sqrt(fmax(rows, cols));
+  else if (a.scale_rule == MUON_SCALE_KELLER) scale = sqrt(fmax(1.0, rows / cols));
+
+  double wdo = sc.wo, doo = sc.o2;  // <W, D O>, ||D O||^2
+  int axis = 0;
+  if (a.equilibrate) {
+    // imbalance = std / mean of the row RMS and of the column RMS vectors
+    double sr = 0, sr2 = 0, scs = 0, sc2 = 0;
+    for (int i = threadIdx.x; i < d.rows; i += kThreads) {
+      const double v = sqrt((double)a.eq_o2[s.eq_off + i] / cols);
+      sr += v;
+      sr2 += v * v;
+    }
+    for (int j = threadIdx.x; j < d.cols; j += kThreads) {
+      const double v = sqrt((double)a.eq_o2[s.eq_off + d.rows + j] / rows);
+      scs += v;
+      sc2 += v * v;
+    }
+    block_sum2(sr, sr2, red);
+    block_sum2(scs, sc2, red);
+    const double mr = sr / rows, mc = scs / cols;
+    const double ir = mr > 0 ? sqrt(fmax(sr2 / rows - mr * mr, 0.0)) / mr : 0.0;
+    const double ic = mc > 0 ? sqrt(fmax(sc2 / cols - mc * mc, 0.0)) / mc : 0.0;
+    axis = (ir >= ic) ? 1 : 2;
+    const double rho = sqrt(sc.o2 / (rows * cols));
+    const int len = axis == 1 ? d.rows : d.cols;
+    const double line = axis == 1 ? cols : rows;
+    const int64_t base = s.eq_off + (axis == 1 ? 0 : d.rows);
+    double dwo = 0, dd = 0;
+    for (int i = threadIdx.x; i < len; i += kThreads) {
+      const double o2 = a.eq_o2[base + i];
+      const double f = rho / (sqrt(o2 / line) + (double)a.eps);
+      dwo += f * (double)a.eq_wo[base + i];
+      dd += f * f * o2;
+      a.eq_o2[base + i] = static_cast<float>(f);  // factors for post_apply
+    }
+    block_sum2(dwo, dd, red);
+    wdo = dwo;
+    doo = dd;
+  }
+  if (threadIdx.x != 0) return;
+  wdo *= scale;                 // <W, O> with O = s*D*O_raw
+  const double oo = scale * scale * doo;
+  double g = 0.0;
+  if (a.mode == MUON_MODE_MUONGS && sc.w2 > 0.0) g = wdo / sc.w2;
+  MatCoef cf;
+  cf.cw = static_cast<float>(1.0 - (double)a.lr * (double)a.wd + (double)a.lr * g);
+  cf.co = static_cast<float>(-(double)a.lr * scale);
+  cf.axis = axis;
+  cf.pad = 0;
+  a.coef[k] = cf;
+  if (a.stats != nullptr) {
+    double ot2 = oo;
+    if (a.mode == MUON_MODE_MUONGS && sc.w2 > 0.0) ot2 = oo - wdo * wdo / sc.w2;
+    muon_stats_t st;
+    st.w_norm = static_cast<float>(sqrt(sc.w2));
+    st.w_dot_o = static_cast<float>(wdo);
+    st.o_norm = static_cast<float>(sqrt(fmax(ot2, 0.0)));
+    st.update_rms = static_cast<float>(sqrt(fmax(ot2, 0.0) / (rows * cols)));
+    st.equil_axis = axis;
+    st.reserved = 0;
+    a.stats[d.orig] = st;
+  }
+}
+
+// ------------------------------------------------------------------ post_apply
+__global__ void __launch_bounds__(kThreads) post_apply_kernel(const ElemArgs a) {
+  __shared__ float tile[kTC][kTR + 1];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int tiles_c = (d.cols + kTC - 1) / kTC;
+  const int r0 = (t / tiles_c) * kTR, c0 = (t % tiles_c) * kTC;
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const int r = r0 + lr, c = c0 + lc;
+  const bool vec = (d.flags & MAT_VEC_OK) != 0;
+  const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+
+  float o[8];
+  load_o_tile(a, d, s, r0, c0, tile, o);
+  if (valid <= 0) return;
+  const float xs = slab_scale(a, k);
+  if (a.ns_only) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] *= xs;
+    if (d.flags & MAT_G_BF16)
+      store8_bf16(reinterpret_cast<uint16_t*>(d.W) + (int64_t)r * d.ld_w + c, vec, valid, o);
+    else
+      store8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, o);
+    return;
+  }
+  const MatCoef cf = a.coef[k];
+  float w[8];
+  float* wp = d.W + (int64_t)r * d.ld_w + c;
+  load8_f32(wp, vec, valid, w);
+  const float rowf = cf.axis == 1 ? a.eq_o2[s.eq_off + r] : 1.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    float f = xs * rowf;
+    if (cf.axis == 2 && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+    w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
+  }
+  store8_f32(wp, vec, valid, w);
+}
+
+}  // namespace
+
+cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
+  if (a.total_tiles <= 0) return cudaSuccess;
+  ingest_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
+  if (a.total_tiles <= 0) return cudaSuccess;
+  post_reduce_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+cudaError_t launch_post_finalize(const ElemArgs& a, cudaStream_t s) {
+  if (a.n <= 0) return cudaSuccess;
+  post_finalize_kernel<<<a.n, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+cudaError_t launch_post_apply(const ElemArgs& a, cudaStream_t s) {
+  if (a.total_tiles <= 0) return cudaSuccess;
+  post_apply_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

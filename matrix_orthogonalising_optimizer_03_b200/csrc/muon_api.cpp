@@ -1,0 +1,790 @@
+// Host side of libmuon: validation, shape grouping (the plan), workspace layout,
+// descriptor upload and the launch sequence of one Muon step.
+//
+// Step order (the update order of "[Deep Learning] Muon — 행렬 업데이트를 직교화하는
+// 옵티마이저", section 3): ingest (momentum, Nesterov, ||U||^2) -> ns_steps x
+// {GRAM, POLY, APPLY} -> post_reduce -> post_finalize -> post_apply.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <new>
+#include <tuple>
+#include <vector>
+
+#include "muon.h"
+#include "muon_internal.h"
+#include "ns_tc.h"
+
+using namespace muon;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kSlabAlign = 1024;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t round_up64(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+struct ClassMaps {
+  CUtensorMap x128[2];  // X slabs, 64 x 128 boxes (K-major operand)
+  CUtensorMap x64[2];   // X slabs, 64 x 64 boxes (MN-major operand of APPLY)
+  CUtensorMap s128;     // S slab
+  CUtensorMap p128;     // P slab
+};
+
+}  // namespace
+
+struct muon_plan_s {
+  bool ns_only = false;
+  int n = 0;
+  muon_hparams_t hp{};
+  bool x_fp32 = false;
+  bool equilibrate = false;
+  std::vector<ClassInfo> classes;
+  std::vector<DevMat> dev;         // plan order
+  std::vector<int64_t> eq_off;     // plan order
+  std::vector<int32_t> tile_prefix;
+  int64_t eq_total = 0;
+  size_t off_scal = 0, off_coef = 0, off_desc = 0, off_slabs = 0, off_tiles = 0;
+  size_t off_eq_o2 = 0, off_eq_wo = 0, ws_bytes = 0;
+  // cached per workspace pointer and device
+  void* ws_cached = nullptr;
+  int dev_cached = -1;
+  int num_sms = 0;
+  std::vector<ClassMaps> maps;
+  // optional per-launch event timing
+  struct ProfRec {
+    cudaEvent_t a, b;
+    int kind;
+    double flops, bytes;
+  };
+  bool prof = false;
+  std::vector<ProfRec> recs;
+  std::vector<cudaEvent_t> event_pool;
+  ~muon_plan_s() {
+    for (const ProfRec& r : recs) {
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
+    }
+    for (cudaEvent_t e : event_pool) cudaEventDestroy(e);
+  }
+};
+
+namespace {
+
+bool valid_enum_hp(const muon_hparams_t* hp) {
+  if (hp->ns_steps < 0 || hp->ns_steps > 64) return false;
+  if (hp->mode != MUON_MODE_MUON && hp->mode != MUON_MODE_MUONGS) return false;
+  if (hp->scale != MUON_SCALE_MOONLIGHT && hp->scale != MUON_SCALE_KELLER &&
+      hp->scale != MUON_SCALE_NONE)
+    return false;
+  const uint32_t known = MUON_NESTEROV | MUON_EQUILIBRATE | MUON_NS_FP32 | MUON_WANT_STATS;
+  if (hp->flags & ~known) return false;
+  if (!(hp->eps >= 0.f) || !std::isfinite(hp->eps)) return false;
+  return true;
+}
+
+struct Interval {
+  uintptr_t lo, hi;
+  bool writable;
+};
+
+// Overlap of a written range with any other range is an error; read-only ranges may overlap.
+bool any_alias(std::vector<Interval>& iv) {
+  std::sort(iv.begin(), iv.end(), [](const Interval& a, const Interval& b) { return a.lo < b.lo; });
+  uintptr_t end_any = 0, end_w = 0;
+  bool first = true;
+  for (const Interval& x : iv) {
+    if (!first) {
+      if (x.lo < end_w) return true;
+      if (x.writable && x.lo < end_any) return true;
+    }
+    first = false;
+    end_any = std::max(end_any, x.hi);
+    if (x.writable) end_w = std::max(end_w, x.hi);
+  }
+  return false;
+}
+
+uintptr_t span_end(const void* p, int64_t rows, int64_t cols, int64_t ld, int esz) {
+  return reinterpret_cast<uintptr_t>(p) + static_cast<uintptr_t>(((rows - 1) * ld + cols) * esz);
+}
+
+muon_status_t check_shape(int64_t rows, int64_t cols) {
+  if (rows < 1 || cols < 1) return MUON_ERR_SHAPE;
+  if (rows > (1 << 24) || cols > (1 << 24) || rows * cols >= (int64_t(1) << 31)) return MUON_ERR_SHAPE;
+  return MUON_OK;
+}
+
+muon_status_t validate_step(const muon_matrix_t* mats, int n, const muon_hparams_t* hp) {
+  if (hp == nullptr || n < 0 || (n > 0 && mats == nullptr)) return MUON_ERR_INVALID_ARG;
+  if (!valid_enum_hp(hp)) return MUON_ERR_INVALID_ARG;
+  std::vector<Interval> iv;
+  iv.reserve(3 * static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    const muon_matrix_t& m = mats[i];
+    if (m.W == nullptr || m.grad == nullptr || m.momentum == nullptr) return MUON_ERR_INVALID_ARG;
+    muon_status_t s = check_shape(m.rows, m.cols);
+    if (s != MUON_OK) return s;
+    if (m.ld_w < m.cols || m.ld_g < m.cols || m.ld_m < m.cols) return MUON_ERR_SHAPE;
+    if (m.w_dtype != MUON_F32) return MUON_ERR_DTYPE;
+    if (m.g_dtype != MUON_F32 && m.g_dtype != MUON_BF16) return MUON_ERR_DTYPE;
+    const int gsz = m.g_dtype == MUON_BF16 ? 2 : 4;
+    if (reinterpret_cast<uintptr_t>(m.W) % 4 || reinterpret_cast<uintptr_t>(m.momentum) % 4 ||
+        reinterpret_cast<uintptr_t>(m.grad) % gsz)
+      return MUON_ERR_INVALID_ARG;
+    iv.push_back({reinterpret_cast<uintptr_t>(m.W), span_end(m.W, m.rows, m.cols, m.ld_w, 4), true});
+    iv.push_back({reinterpret_cast<uintptr_t>(m.momentum),
+                  span_end(m.momentum, m.rows, m.cols, m.ld_m, 4), true});
+    iv.push_back({reinterpret_cast<uintptr_t>(m.grad), span_end(m.grad, m.rows, m.cols, m.ld_g, gsz),
+                  false});
+  }
+  if (any_alias(iv)) return MUON_ERR_ALIAS;
+  return MUON_OK;
+}
+
+muon_status_t validate_ns(const muon_ns_matrix_t* mats, int n, const muon_hparams_t* hp) {
+  if (hp == nullptr || n < 0 || (n > 0 && mats == nullptr)) return MUON_ERR_INVALID_ARG;
+  if (!valid_enum_hp(hp)) return MUON_ERR_INVALID_ARG;
+  std::vector<Interval> iv;
+  for (int i = 0; i < n; ++i) {
+    const muon_ns_matrix_t& m = mats[i];
+    if (m.X == nullptr || m.O == nullptr) return MUON_ERR_INVALID_ARG;
+    muon_status_t s = check_shape(m.rows, m.cols);
+    if (s != MUON_OK) return s;
+    if (m.ld_x < m.cols || m.ld_o < m.cols) return MUON_ERR_SHAPE;
+    if (m.dtype != MUON_F32 && m.dtype != MUON_BF16) return MUON_ERR_DTYPE;
+    const int esz = m.dtype == MUON_BF16 ? 2 : 4;
+    if (reinterpret_cast<uintptr_t>(m.X) % esz || reinterpret_cast<uintptr_t>(m.O) % esz)
+      return MUON_ERR_INVALID_ARG;
+    iv.push_back({reinterpret_cast<uintptr_t>(m.O), span_end(m.O, m.rows, m.cols, m.ld_o, esz), true});
+    iv.push_back({reinterpret_cast<uintptr_t>(m.X), span_end(m.X, m.rows, m.cols, m.ld_x, esz), false});
+  }
+  if (any_alias(iv)) return MUON_ERR_ALIAS;
+  return MUON_OK;
+}
+
+// Groups matrices by oriented shape and lays out the workspace.
+void build_plan(muon_plan_s* p) {
+  const int n = p->n;
+  const bool x_fp32 = p->x_fp32;
+  const int esz = x_fp32 ? 4 : 2;
+  // class key: (m, n) oriented; heavier classes first (longer reductions first
+  // in the persistent tile order)
+  std::map<std::pair<int, int>, std::vector<int>> groups;
+  for (int i = 0; i < n; ++i) {
+    const int r = p->dev[i].rows, c = p->dev[i].cols;
+    groups[{std::min(r, c), std::max(r, c)}].push_back(i);
+  }
+  std::vector<std::pair<std::pair<int, int>, std::vector<int>>> order(groups.begin(), groups.end());
+  std::stable_sort(order.begin(), order.end(), [](const auto& a, const auto& b) {
+    const double wa = double(a.first.first) * a.first.first * a.first.second;
+    const double wb = double(b.first.first) * b.first.first * b.first.second;
+    return wa > wb;
+  });
+  std::vector<DevMat> sorted;
+  std::vector<int64_t> eq_off;
+  sorted.reserve(n);
+  p->classes.clear();
+  int64_t eq_total = 0;
+  for (auto& g : order) {
+    ClassInfo ci{};
+    ci.m = g.first.first;
+    ci.n = g.first.second;
+    ci.count = static_cast<int32_t>(g.second.size());
+    ci.first = static_cast<int32_t>(sorted.size());
+    ci.ldx = static_cast<int32_t>(round_up64(ci.n, 64));
+    ci.lds = static_cast<int32_t>(round_up64(ci.m, 64));
+    ci.xbytes = int64_t(ci.m) * ci.ldx * esz;
+    ci.sbytes = int64_t(ci.m) * ci.lds * esz;
+    for (int idx : g.second) {
+      sorted.push_back(p->dev[idx]);
+      eq_off.push_back(eq_total);
+      eq_total += p->dev[idx].rows + p->dev[idx].cols;
+    }
+    p->classes.push_back(ci);
+  }
+  p->dev.swap(sorted);
+  p->eq_off.swap(eq_off);
+  p->eq_total = p->equilibrate ? eq_total : 0;
+  // elementwise tiles
+  p->tile_prefix.assign(n + 1, 0);
+  for (int i = 0; i < n; ++i) {
+    const int64_t t = int64_t((p->dev[i].rows + kElemTileR - 1) / kElemTileR) *
+                      ((p->dev[i].cols + kElemTileC - 1) / kElemTileC);
+    p->tile_prefix[i + 1] = static_cast<int32_t>(p->tile_prefix[i] + t);
+  }
+  // workspace layout
+  size_t off = align_up(sizeof(WsHeader), kAlign);
+  p->off_scal = off;   off = align_up(off + sizeof(MatScalars) * n, kAlign);
+  p->off_coef = off;   off = align_up(off + sizeof(MatCoef) * n, kAlign);
+  p->off_desc = off;   off = align_up(off + sizeof(DevMat) * n, kAlign);
+  p->off_slabs = off;  off = align_up(off + sizeof(DevSlab) * n, kAlign);
+  p->off_tiles = off;  off = align_up(off + sizeof(int32_t) * (n + 1), kAlign);
+  p->off_eq_o2 = off;  off = align_up(off + sizeof(float) * p->eq_total, kAlign);
+  p->off_eq_wo = off;  off = align_up(off + sizeof(float) * p->eq_total, kAlign);
+  off = align_up(off, kSlabAlign);
+  const bool two_x = p->hp.ns_steps > 0;
+  for (ClassInfo& ci : p->classes) {
+    ci.off_x[0] = static_cast<int64_t>(off);
+    off = align_up(off + ci.xbytes * ci.count, kSlabAlign);
+    if (two_x) {
+      ci.off_x[1] = static_cast<int64_t>(off);
+      off = align_up(off + ci.xbytes * ci.count, kSlabAlign);
+    } else {
+      ci.off_x[1] = ci.off_x[0];
+    }
+    if (p->hp.ns_steps > 0) {
+      ci.off_s = static_cast<int64_t>(off);
+      off = align_up(off + ci.sbytes * ci.count, kSlabAlign);
+      ci.off_p = static_cast<int64_t>(off);
+      off = align_up(off + ci.sbytes * ci.count, kSlabAlign);
+    } else {
+      ci.off_s = ci.off_p = ci.off_x[0];
+    }
+  }
+  p->ws_bytes = off;
+}
+
+int32_t vec_flag(const void* a, const void* b, const void* c, int64_t la, int64_t lb, int64_t lc,
+                 int ea, int eb, int ec) {
+  auto ok = [](const void* ptr, int64_t ld, int esz) {
+    if (ptr == nullptr) return true;
+    return reinterpret_cast<uintptr_t>(ptr) % 16 == 0 && (ld * esz) % 16 == 0;
+  };
+  return (ok(a, la, ea) && ok(b, lb, eb) && ok(c, lc, ec)) ? MAT_VEC_OK : 0;
+}
+
+muon_plan_s* make_step_plan(const muon_matrix_t* mats, int n, const muon_hparams_t* hp) {
+  muon_plan_s* p = new (std::nothrow) muon_plan_s();
+  if (p == nullptr) return nullptr;
+  p->ns_only = false;
+  p->n = n;
+  p->hp = *hp;
+  p->x_fp32 = (hp->flags & MUON_NS_FP32) != 0;
+  p->equilibrate = (hp->flags & MUON_EQUILIBRATE) != 0;
+  p->dev.resize(n);
+  for (int i = 0; i < n; ++i) {
+    const muon_matrix_t& m = mats[i];
+    DevMat d{};
+    d.W = static_cast<float*>(m.W);
+    d.G = m.grad;
+    d.M = static_cast<float*>(m.momentum);
+    d.ld_w = m.ld_w;
+    d.ld_g = m.ld_g;
+    d.ld_m = m.ld_m;
+    d.rows = static_cast<int32_t>(m.rows);
+    d.cols = static_cast<int32_t>(m.cols);
+    const bool gb = m.g_dtype == MUON_BF16;
+    d.flags = (m.rows > m.cols ? MAT_TRANSPOSED : 0) | (gb ? MAT_G_BF16 : 0) |
+              vec_flag(m.W, m.grad, m.momentum, m.ld_w, m.ld_g, m.ld_m, 4, gb ? 2 : 4, 4);
+    d.orig = i;
+    p->dev[i] = d;
+  }
+  build_plan(p);
+  return p;
+}
+
+muon_plan_s* make_ns_plan(const muon_ns_matrix_t* mats, int n, const muon_hparams_t* hp) {
+  muon_plan_s* p = new (std::nothrow) muon_plan_s();
+  if (p == nullptr) return nullptr;
+  p->ns_only = true;
+  p->n = n;
+  p->hp = *hp;
+  p->x_fp32 = (hp->flags & MUON_NS_FP32) != 0;
+  p->equilibrate = false;
+  p->dev.resize(n);
+  for (int i = 0; i < n; ++i) {
+    const muon_ns_matrix_t& m = mats[i];
+    const bool b = m.dtype == MUON_BF16;
+    DevMat d{};
+    d.W = static_cast<float*>(m.O);  // output
+    d.G = m.X;                        // input
+    d.M = nullptr;
+    d.ld_w = m.ld_o;
+    d.ld_g = m.ld_x;
+    d.ld_m = 0;
+    d.rows = static_cast<int32_t>(m.rows);
+    d.cols = static_cast<int32_t>(m.cols);
+    d.flags = (m.rows > m.cols ? MAT_TRANSPOSED : 0) | (b ? MAT_G_BF16 : 0) |
+              vec_flag(m.O, m.X, nullptr, m.ld_o, m.ld_x, 0, b ? 2 : 4, b ? 2 : 4, 4);
+    d.orig = i;
+    p->dev[i] = d;
+  }
+  build_plan(p);
+  return p;
+}
+
+struct DeviceInfo {
+  bool checked = false;
+  bool ok = false;
+  int num_sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+muon_status_t current_device(int* dev, int* num_sms) {
+  if (cudaGetDevice(dev) != cudaSuccess) return MUON_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return MUON_ERR_UNSUPPORTED;
+  DeviceInfo& di = g_dev[*dev];
+  if (!di.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
+      return MUON_ERR_CUDA;
+    di.ok = (major == 10 && minor == 0);
+    di.num_sms = sms;
+    di.checked = true;
+  }
+  if (!di.ok) return MUON_ERR_UNSUPPORTED;
+  *num_sms = di.num_sms;
+  return MUON_OK;
+}
+
+// Binds the plan to a workspace: absolute slab pointers, tensor maps, and the
+// device copy of the descriptor tables.
+muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int n = p->n;
+  const int steps = p->hp.ns_steps;
+  std::vector<DevSlab> slabs(n);
+  for (size_t c = 0; c < p->classes.size(); ++c) {
+    const ClassInfo& ci = p->classes[c];
+    for (int i = 0; i < ci.count; ++i) {
+      DevSlab s{};
+      s.x0 = base + ci.off_x[0] + ci.xbytes * i;
+      s.xf = base + ci.off_x[steps % 2] + ci.xbytes * i;
+      s.ldx = ci.ldx;
+      s.cls = static_cast<int32_t>(c);
+      s.eq_off = p->eq_off[ci.first + i];
+      slabs[ci.first + i] = s;
+    }
+  }
+  p->maps.clear();
+  if (!p->x_fp32 && steps > 0) {
+    p->maps.resize(p->classes.size());
+    for (size_t c = 0; c < p->classes.size(); ++c) {
+      const ClassInfo& ci = p->classes[c];
+      ClassMaps& cm = p->maps[c];
+      bool ok = true;
+      for (int b = 0; b < 2; ++b) {
+        ok = ok && encode_slab_map_bf16(&cm.x128[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 128);
+        ok = ok && encode_slab_map_bf16(&cm.x64[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 64);
+      }
+      ok = ok && encode_slab_map_bf16(&cm.s128, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 128);
+      ok = ok && encode_slab_map_bf16(&cm.p128, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 128);
+      if (!ok) return MUON_ERR_CUDA;
+    }
+  }
+  // one upload of [desc | slabs | tiles]
+  const size_t lo = p->off_desc, hi = p->off_tiles + sizeof(int32_t) * (n + 1);
+  std::vector<uint8_t> host(hi - lo, 0);
+  std::memcpy(host.data() + (p->off_desc - lo), p->dev.data(), sizeof(DevMat) * n);
+  std::memcpy(host.data() + (p->off_slabs - lo), slabs.data(), sizeof(DevSlab) * n);
+  std::memcpy(host.data() + (p->off_tiles - lo), p->tile_prefix.data(), sizeof(int32_t) * (n + 1));
+  if (cudaMemcpyAsync(base + lo, host.data(), host.size(), cudaMemcpyHostToDevice, stream) !=
+      cudaSuccess)
+    return MUON_ERR_CUDA;
+  // a fresh workspace starts with a clear device error word
+  if (cudaMemsetAsync(base, 0, sizeof(WsHeader), stream) != cudaSuccess) return MUON_ERR_CUDA;
+  p->ws_cached = ws;
+  p->dev_cached = dev;
+  return MUON_OK;
+}
+
+void fill_class_args(const muon_plan_s* p, uint8_t* base, size_t c, int phase, int it,
+                     NsClassArgs* k, int bm, int bn, int bk) {
+  const ClassInfo& ci = p->classes[c];
+  const int esz = p->x_fp32 ? 4 : 2;
+  k->m = ci.m;
+  k->n = ci.n;
+  k->count = ci.count;
+  k->first = ci.first;
+  k->ldx = ci.ldx;
+  k->lds = ci.lds;
+  k->xstride = ci.xbytes / esz;
+  k->sstride = ci.sbytes / esz;
+  k->x_in = base + ci.off_x[it % 2];
+  k->x_out = base + ci.off_x[(it + 1) % 2];
+  k->s = base + ci.off_s;
+  k->p = base + ci.off_p;
+  const int ncols = phase == PH_APPLY ? ci.n : ci.m;
+  k->tiles_i = (ci.m + bm - 1) / bm;
+  k->tiles_j = (ncols + bn - 1) / bn;
+  k->tiles_per_mat = phase == PH_APPLY ? k->tiles_i * k->tiles_j : k->tiles_i * (k->tiles_i + 1) / 2;
+  const int K = phase == PH_GRAM ? ci.n : ci.m;
+  k->k_blocks = (K + bk - 1) / bk;
+}
+
+enum ProfKind { PK_INGEST = 0, PK_GRAM, PK_POLY, PK_APPLY, PK_REDUCE, PK_FINALIZE, PK_POST, PK_COUNT };
+const char* const kProfNames[PK_COUNT] = {"ingest", "ns_gram", "ns_poly", "ns_apply",
+                                          "post_reduce", "post_finalize", "post_apply"};
+constexpr size_t kMaxProfRecs = 1 << 16;
+
+cudaEvent_t prof_event(muon_plan_s* p) {
+  if (!p->event_pool.empty()) {
+    cudaEvent_t e = p->event_pool.back();
+    p->event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+// Brackets one launch with events when profiling is on.
+struct ProfScope {
+  muon_plan_s* p;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  ProfScope(muon_plan_s* plan, cudaStream_t stream) : p(plan), s(stream) {
+    if (p->prof && p->recs.size() < kMaxProfRecs) {
+      a = prof_event(p);
+      if (a != nullptr && cudaEventRecord(a, s) != cudaSuccess) {
+        p->event_pool.push_back(a);
+        a = nullptr;
+      }
+    }
+  }
+  void done(int kind, double flops, double bytes) {
+    if (a == nullptr) return;
+    cudaEvent_t b = prof_event(p);
+    if (b == nullptr || cudaEventRecord(b, s) != cudaSuccess) {
+      p->event_pool.push_back(a);
+      if (b) p->event_pool.push_back(b);
+      a = nullptr;
+      return;
+    }
+    p->recs.push_back({a, b, kind, flops, bytes});
+    a = nullptr;
+  }
+};
+
+double class_phase_flops(const ClassInfo& ci, int phase) {
+  const double m = ci.m, n = ci.n;
+  double f = phase == PH_GRAM ? m * (m + 1) * n : (phase == PH_POLY ? m * m * (m + 1) : 2 * m * m * n);
+  return f * ci.count;
+}
+
+double elem_bytes(const muon_plan_s* p, int kind) {
+  const int ex = p->x_fp32 ? 4 : 2;
+  double total = 0;
+  for (const DevMat& d : p->dev) {
+    const double e = double(d.rows) * d.cols;
+    const int eg = (d.flags & MAT_G_BF16) ? 2 : 4;
+    if (kind == PK_INGEST) total += e * (p->ns_only ? eg + ex : eg + 8 + ex);
+    else if (kind == PK_REDUCE) total += e * (4 + ex);
+    else if (kind == PK_POST) total += e * (p->ns_only ? eg + ex : 8 + ex);
+  }
+  return total;
+}
+
+muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* stats,
+                       cudaStream_t stream) {
+  if (p->n == 0) return MUON_OK;
+  if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < p->ws_bytes)
+    return MUON_ERR_WORKSPACE;
+  int dev = 0, num_sms = 0;
+  muon_status_t st = current_device(&dev, &num_sms);
+  if (st != MUON_OK) return st;
+  p->num_sms = num_sms;
+  if (p->ws_cached != ws || p->dev_cached != dev) {
+    st = bind_workspace(p, ws, dev, stream);
+    if (st != MUON_OK) return st;
+  }
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int n = p->n;
+  const muon_hparams_t& hp = p->hp;
+  if (cudaMemsetAsync(base + p->off_scal, 0, sizeof(MatScalars) * n, stream) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (p->eq_total > 0) {
+    if (cudaMemsetAsync(base + p->off_eq_o2, 0, p->off_eq_wo - p->off_eq_o2 + sizeof(float) * p->eq_total,
+                        stream) != cudaSuccess)
+      return MUON_ERR_CUDA;
+  }
+  ElemArgs ea{};
+  ea.mats = reinterpret_cast<const DevMat*>(base + p->off_desc);
+  ea.slabs = reinterpret_cast<const DevSlab*>(base + p->off_slabs);
+  ea.tile_prefix = reinterpret_cast<const int32_t*>(base + p->off_tiles);
+  ea.n = n;
+  ea.total_tiles = p->tile_prefix[n];
+  ea.scal = reinterpret_cast<MatScalars*>(base + p->off_scal);
+  ea.coef = reinterpret_cast<MatCoef*>(base + p->off_coef);
+  ea.eq_o2 = reinterpret_cast<float*>(base + p->off_eq_o2);
+  ea.eq_wo = reinterpret_cast<float*>(base + p->off_eq_wo);
+  ea.stats = p->ns_only ? nullptr : stats;
+  ea.err = reinterpret_cast<uint32_t*>(base);
+  ea.mu = hp.momentum;
+  ea.lr = hp.lr;
+  ea.wd = hp.weight_decay;
+  ea.eps = hp.eps;
+  ea.scale_k = hp.scale_k;
+  ea.scale_rule = hp.scale;
+  ea.mode = hp.mode;
+  ea.nesterov = (hp.flags & MUON_NESTEROV) ? 1 : 0;
+  ea.ns_only = p->ns_only ? 1 : 0;
+  ea.x_fp32 = p->x_fp32 ? 1 : 0;
+  ea.equilibrate = p->equilibrate ? 1 : 0;
+  ea.xs_from_u2 = hp.ns_steps == 0 ? 1 : 0;
+
+  {
+    ProfScope ps(p, stream);
+    if (launch_ingest(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    ps.done(PK_INGEST, 0.0, elem_bytes(p, PK_INGEST));
+  }
+
+  // Newton-Schulz phases, at most kMaxClassesPerLaunch classes per launch
+  const int nc = static_cast<int>(p->classes.size());
+  for (int it = 0; it < hp.ns_steps; ++it) {
+    for (int phase = PH_GRAM; phase <= PH_APPLY; ++phase) {
+      for (int c0 = 0; c0 < nc; c0 += kMaxClassesPerLaunch) {
+        const int cn = std::min(kMaxClassesPerLaunch, nc - c0);
+        if (p->x_fp32) {
+          NsPhaseArgs a{};
+          a.num_classes = cn;
+          a.phase = phase;
+          a.a = hp.ns_coeffs[0];
+          a.b = hp.ns_coeffs[1];
+          a.c = hp.ns_coeffs[2];
+          a.first_iter = it == 0 ? 1 : 0;
+          a.eps = hp.eps;
+          a.scal = ea.scal;
+          a.err = ea.err;
+          int tiles = 0;
+          for (int c = 0; c < cn; ++c) {
+            fill_class_args(p, base, c0 + c, phase, it, &a.cls[c], 64, 64, 16);
+            a.tile_base[c] = tiles;
+            tiles += a.cls[c].count * a.cls[c].tiles_per_mat;
+          }
+          a.tile_base[cn] = tiles;
+          ProfScope ps(p, stream);
+          if (launch_ns_phase_simt(a, stream) != cudaSuccess) return MUON_ERR_CUDA;
+          double fl = 0;
+          for (int c = 0; c < cn; ++c) fl += class_phase_flops(p->classes[c0 + c], phase);
+          ps.done(PK_GRAM + phase, fl, 0.0);
+        } else {
+          TcParams P;
+          std::memset(&P, 0, sizeof(P));
+          NsPhaseArgs& a = P.args;
+          a.num_classes = cn;
+          a.phase = phase;
+          a.a = hp.ns_coeffs[0];
+          a.b = hp.ns_coeffs[1];
+          a.c = hp.ns_coeffs[2];
+          a.first_iter = it == 0 ? 1 : 0;
+          a.eps = hp.eps;
+          a.scal = ea.scal;
+          a.err = ea.err;
+          int tiles = 0;
+          for (int c = 0; c < cn; ++c) {
+            const ClassMaps& cm = p->maps[c0 + c];
+            fill_class_args(p, base, c0 + c, phase, it, &a.cls[c], tc_block_m(), tc_block_n(phase),
+                            tc_block_k());
+            a.tile_base[c] = tiles;
+            tiles += a.cls[c].count * a.cls[c].tiles_per_mat;
+            if (phase == PH_GRAM) {
+              P.ta[c] = cm.x128[it % 2];
+              P.tb[c] = cm.x128[it % 2];
+            } else if (phase == PH_POLY) {
+              P.ta[c] = cm.s128;
+              P.tb[c] = cm.s128;
+            } else {
+              P.ta[c] = cm.p128;
+              P.tb[c] = cm.x64[it % 2];
+            }
+          }
+          a.tile_base[cn] = tiles;
+          ProfScope ps(p, stream);
+          if (launch_ns_phase_tc(P, num_sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
+          double fl = 0;
+          for (int c = 0; c < cn; ++c) fl += class_phase_flops(p->classes[c0 + c], phase);
+          ps.done(PK_GRAM + phase, fl, 0.0);
+        }
+      }
+    }
+  }
+
+  if (!p->ns_only) {
+    const bool need_reduce = hp.mode == MUON_MODE_MUONGS || p->equilibrate || stats != nullptr;
+    if (need_reduce) {
+      ProfScope ps(p, stream);
+      if (launch_post_reduce(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
+      ps.done(PK_REDUCE, 0.0, elem_bytes(p, PK_REDUCE));
+    }
+    ProfScope ps(p, stream);
+    if (launch_post_finalize(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    ps.done(PK_FINALIZE, 0.0, 0.0);
+  }
+  ProfScope ps(p, stream);
+  if (launch_post_apply(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
+  ps.done(PK_POST, 0.0, elem_bytes(p, PK_POST));
+  return MUON_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int muon_abi_version(void) { return MUON_ABI_VERSION; }
+
+const char* muon_status_string(muon_status_t s) {
+  switch (s) {
+    case MUON_OK: return "MUON_OK";
+    case MUON_ERR_INVALID_ARG: return "MUON_ERR_INVALID_ARG";
+    case MUON_ERR_SHAPE: return "MUON_ERR_SHAPE";
+    case MUON_ERR_DTYPE: return "MUON_ERR_DTYPE";
+    case MUON_ERR_ALIAS: return "MUON_ERR_ALIAS";
+    case MUON_ERR_WORKSPACE: return "MUON_ERR_WORKSPACE";
+    case MUON_ERR_CUDA: return "MUON_ERR_CUDA";
+    case MUON_ERR_TIMEOUT: return "MUON_ERR_TIMEOUT";
+    case MUON_ERR_UNSUPPORTED: return "MUON_ERR_UNSUPPORTED";
+  }
+  return "MUON_ERR_UNKNOWN";
+}
+
+muon_status_t muon_hparams_default(muon_hparams_t* hp) {
+  if (hp == nullptr) return MUON_ERR_INVALID_ARG;
+  std::memset(hp, 0, sizeof(*hp));
+  hp->lr = 0.02f;
+  hp->momentum = 0.95f;
+  hp->weight_decay = 0.f;
+  hp->ns_coeffs[0] = 3.4445f;
+  hp->ns_coeffs[1] = -4.7750f;
+  hp->ns_coeffs[2] = 2.0315f;
+  hp->ns_steps = 5;
+  hp->eps = 1e-7f;
+  hp->mode = MUON_MODE_MUON;
+  hp->scale = MUON_SCALE_MOONLIGHT;
+  hp->scale_k = 0.2f;
+  hp->flags = MUON_NESTEROV;
+  return MUON_OK;
+}
+
+muon_status_t muon_validate(const muon_matrix_t* mats, int n, const muon_hparams_t* hp) {
+  return validate_step(mats, n, hp);
+}
+
+size_t muon_workspace_size(const muon_matrix_t* mats, int n, const muon_hparams_t* hp) {
+  if (validate_step(mats, n, hp) != MUON_OK) return 0;
+  muon_plan_s* p = make_step_plan(mats, n, hp);
+  if (p == nullptr) return 0;
+  const size_t s = p->ws_bytes;
+  delete p;
+  return s;
+}
+
+muon_status_t muon_step_batched(const muon_matrix_t* mats, int n, const muon_hparams_t* hp,
+                                void* workspace, size_t ws_bytes, muon_stats_t* stats_dev,
+                                void* stream) {
+  muon_status_t st = validate_step(mats, n, hp);
+  if (st != MUON_OK || n == 0) return st;
+  muon_plan_s* p = make_step_plan(mats, n, hp);
+  if (p == nullptr) return MUON_ERR_INVALID_ARG;
+  st = run_plan(p, workspace, ws_bytes, stats_dev, static_cast<cudaStream_t>(stream));
+  delete p;
+  return st;
+}
+
+muon_status_t muon_plan_create(const muon_matrix_t* mats, int n, const muon_hparams_t* hp,
+                               muon_plan_t* out) {
+  if (out == nullptr) return MUON_ERR_INVALID_ARG;
+  *out = nullptr;
+  muon_status_t st = validate_step(mats, n, hp);
+  if (st != MUON_OK) return st;
+  muon_plan_s* p = make_step_plan(mats, n, hp);
+  if (p == nullptr) return MUON_ERR_INVALID_ARG;
+  *out = p;
+  return MUON_OK;
+}
+
+size_t muon_plan_workspace_size(muon_plan_t plan) { return plan ? plan->ws_bytes : 0; }
+
+muon_status_t muon_plan_set_hparams(muon_plan_t plan, const muon_hparams_t* hp) {
+  if (plan == nullptr || hp == nullptr || !valid_enum_hp(hp)) return MUON_ERR_INVALID_ARG;
+  const uint32_t layout = MUON_NS_FP32 | MUON_EQUILIBRATE;
+  if ((hp->flags & layout) != (plan->hp.flags & layout)) return MUON_ERR_INVALID_ARG;
+  if ((hp->ns_steps == 0) != (plan->hp.ns_steps == 0)) return MUON_ERR_INVALID_ARG;
+  const bool parity_changed = (hp->ns_steps % 2) != (plan->hp.ns_steps % 2);
+  plan->hp = *hp;
+  if (parity_changed) plan->ws_cached = nullptr;  // the result slab moved: re-upload
+  return MUON_OK;
+}
+
+muon_status_t muon_plan_step(muon_plan_t plan, void* workspace, size_t ws_bytes,
+                             muon_stats_t* stats_dev, void* stream) {
+  if (plan == nullptr) return MUON_ERR_INVALID_ARG;
+  return run_plan(plan, workspace, ws_bytes, stats_dev, static_cast<cudaStream_t>(stream));
+}
+
+void muon_plan_destroy(muon_plan_t plan) { delete plan; }
+
+muon_status_t muon_plan_profile_enable(muon_plan_t plan, int enable) {
+  if (plan == nullptr) return MUON_ERR_INVALID_ARG;
+  plan->prof = enable != 0;
+  return MUON_OK;
+}
+
+int muon_plan_profile_read(muon_plan_t plan, muon_profile_entry_t* out, int max_entries) {
+  if (plan == nullptr || (out == nullptr && max_entries > 0) || max_entries < 0) return -1;
+  muon_profile_entry_t acc[PK_COUNT];
+  std::memset(acc, 0, sizeof(acc));
+  for (int k = 0; k < PK_COUNT; ++k) std::strncpy(acc[k].name, kProfNames[k], sizeof(acc[k].name) - 1);
+  bool ok = true;
+  for (const auto& r : plan->recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+      ok = false;
+    acc[r.kind].launches += 1;
+    acc[r.kind].total_ms += ms;
+    acc[r.kind].flops += r.flops;
+    acc[r.kind].bytes += r.bytes;
+    plan->event_pool.push_back(r.a);
+    plan->event_pool.push_back(r.b);
+  }
+  plan->recs.clear();
+  if (!ok) return -1;
+  const int nw = std::min(max_entries, static_cast<int>(PK_COUNT));
+  for (int k = 0; k < nw; ++k) out[k] = acc[k];
+  return nw;
+}
+
+size_t muon_ns_workspace_size(const muon_ns_matrix_t* mats, int n, const muon_hparams_t* hp) {
+  if (validate_ns(mats, n, hp) != MUON_OK) return 0;
+  muon_plan_s* p = make_ns_plan(mats, n, hp);
+  if (p == nullptr) return 0;
+  const size_t s = p->ws_bytes;
+  delete p;
+  return s;
+}
+
+muon_status_t muon_newton_schulz_batched(const muon_ns_matrix_t* mats, int n,
+                                         const muon_hparams_t* hp, void* workspace,
+                                         size_t ws_bytes, void* stream) {
+  muon_status_t st = validate_ns(mats, n, hp);
+  if (st != MUON_OK || n == 0) return st;
+  muon_plan_s* p = make_ns_plan(mats, n, hp);
+  if (p == nullptr) return MUON_ERR_INVALID_ARG;
+  st = run_plan(p, workspace, ws_bytes, nullptr, static_cast<cudaStream_t>(stream));
+  delete p;
+  return st;
+}
+
+muon_status_t muon_query_device_status(void* workspace, void* stream) {
+  if (workspace == nullptr) return MUON_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MUON_ERR_CUDA;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MUON_ERR_CUDA;
+  if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MUON_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MUON_ERR_CUDA;
+  return word == 0 ? MUON_OK : static_cast<muon_status_t>(word);
+}
+
+}  // extern "C"

@@ -155,3 +155,10 @@ def ns_flops(rows: int, cols: int, steps: int = 5) -> int:
 
 def workload_ns_flops(w: Workload, steps: int = 5) -> int:
     return sum(ns_flops(r, c, steps) * k for r, c, k, _ in w.layout)
+
+
+def normal(rows: int, cols: int, seed: int, std: float, bf16: bool = False) -> np.ndarray:
+    """A seeded N(0, std^2) float32 matrix outside the named shape sets (test cases)."""
+    g = np.random.Generator(np.random.Philox(np.random.SeedSequence([BASE_SEED, 1000, seed])))
+    x = g.standard_normal((rows, cols), dtype=np.float32) * np.float32(std)
+    return bf16_round(x) if bf16 else x

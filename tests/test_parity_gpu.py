@@ -1,0 +1,148 @@
+"""GPU parity of the CUDA path (through the C ABI) against the float64 oracle.
+
+Tolerances (relative Frobenius error per matrix): 1e-4 for the fp32 Newton-Schulz
+path, 3e-2 for the bf16 tensor-core path; checked on W_t, M_t and dW_t.
+"""
+import numpy as np
+import pytest
+
+from oracle import muon_oracle as orc
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def env(lib):
+    import torch
+    from matrix_orthogonalising_optimizer_03_b200 import binding as B
+    return B, torch
+
+
+# ------------------------------------------------------------------ Newton-Schulz only
+def _ns_gpu(B, torch, xs, hp, dtype):
+    X = [torch.tensor(x, dtype=torch.float32, device="cuda").to(dtype) for x in xs]
+    O = [torch.empty_like(x) for x in X]
+    ws = B.newton_schulz(X, O, hp)
+    torch.cuda.synchronize()
+    assert B.load().muon_query_device_status(ws.data_ptr(), None) == 0
+    return [o.double().cpu().numpy() for o in O]
+
+
+SMALL = [(1, 1), (1, 40), (40, 1), (17, 33), (33, 17), (64, 64), (128, 256), (256, 128),
+         (129, 130), (200, 700), (700, 200), (320, 512), (512, 320)]
+
+
+@pytest.mark.parametrize("coeffs,tol", [((1.0, 0.0, 0.0), 1e-2), ((0.0, 1.0, 0.0), 1e-2),
+                                        ((0.0, 0.0, 1.0), 2e-2)])
+def test_tensor_core_phases_isolated(env, coeffs, tol):
+    """One iteration with (a,b,c) = e1, e2, e3 isolates a*X (APPLY epilogue), S X (GRAM
+    then APPLY) and S^2 X (GRAM, POLY, APPLY): each against the literal recurrence."""
+    B, torch = env
+    shapes = [(17, 33), (128, 256), (129, 130), (320, 512), (512, 320), (200, 700)]
+    xs = [H.seeded_bf16(r, c, 10 + i, 1.0) for i, (r, c) in enumerate(shapes)]
+    hp = B.hparams(ns_coeffs=coeffs, ns_steps=1)
+    got = _ns_gpu(B, torch, xs, hp, torch.bfloat16)
+    for x, g in zip(xs, got):
+        want = orc.orthogonalise(x.astype(np.float64), orc.HParams(ns_coeffs=coeffs, ns_steps=1))
+        assert H.rel(g, want) <= tol, (x.shape, H.rel(g, want))
+
+
+@pytest.mark.parametrize("fp32", [True, False])
+def test_newton_schulz_small_shapes(env, fp32):
+    B, torch = env
+    xs = [H.seeded(r, c, 100 + i, 1e-3) for i, (r, c) in enumerate(SMALL)]
+    if not fp32:
+        xs = [H.seeded_bf16(r, c, 100 + i, 1e-3) for i, (r, c) in enumerate(SMALL)]
+    hp = B.hparams(ns_fp32=fp32)
+    got = _ns_gpu(B, torch, xs, hp, torch.float32 if fp32 else torch.bfloat16)
+    tol = H.TOL_FP32 if fp32 else H.TOL_BF16
+    for x, g in zip(xs, got):
+        want = orc.orthogonalise(x.astype(np.float64), orc.HParams())
+        # a bf16 output adds its own rounding (2^-9 relative) on top of the path's error
+        assert H.rel(g, want) <= tol, (x.shape, H.rel(g, want))
+
+
+def test_newton_schulz_zero_steps_and_zero_input(env):
+    B, torch = env
+    xs = [H.seeded(48, 80, 7, 1.0), np.zeros((16, 24), np.float32)]
+    got = _ns_gpu(B, torch, xs, B.hparams(ns_steps=0, ns_fp32=True), torch.float32)
+    assert H.rel(got[0], orc.frobenius_normalise(xs[0].astype(np.float64))) <= 1e-6
+    assert not np.any(got[1])
+    got = _ns_gpu(B, torch, [xs[1]], B.hparams(), torch.bfloat16)
+    assert not np.any(got[0])
+
+
+# ------------------------------------------------------------------ whole step
+@pytest.mark.parametrize("mode", ["muon", "muongs"])
+def test_single_128x256_fp32_ten_steps(env, mode):
+    """The single-matrix case: W 128x256 ~ N(0, 0.02^2), grads N(0, 1e-3^2) fp32, zero
+    momentum, lr 0.02, wd 0.1, 0.2*sqrt(256) scale, 10 steps, fp32 path, 1e-4."""
+    B, torch = env
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+    w = wl.WORKLOADS["single_128x256"]
+    spec = w.matrices()[0]
+    W0 = [wl.weight(w, spec)]
+    grads = [[wl.grad(w, spec, t)] for t in range(10)]
+    hp = H.gpu_hp(B, mode=mode, wd=0.1, ns_fp32=True)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.float32)
+    worst = H.compare_runs(gpu, W0, grads, H.oracle_hp(mode=mode, wd=0.1), H.TOL_FP32)
+    assert worst["dW"] <= H.TOL_FP32
+
+
+STEP_SHAPES = [(17, 33), (33, 17), (128, 256), (256, 128), (200, 700), (320, 512), (512, 320),
+               (384, 384)]
+
+
+@pytest.mark.parametrize("mode,wd,eq", [("muongs", 0.0, False), ("muon", 0.1, False),
+                                        ("muon", 0.1, True), ("muongs", 0.1, True)])
+def test_bf16_step_mixed_shapes_ten_steps(env, mode, wd, eq):
+    B, torch = env
+    W0 = [H.seeded(r, c, 300 + i, 0.02) for i, (r, c) in enumerate(STEP_SHAPES)]
+    grads = [[H.seeded_bf16(r, c, 1000 * (t + 1) + i, 1e-3) for i, (r, c) in enumerate(STEP_SHAPES)]
+             for t in range(10)]
+    hp = H.gpu_hp(B, mode=mode, wd=wd, equilibrate=eq)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.bfloat16)
+    H.compare_runs(gpu, W0, grads, H.oracle_hp(mode=mode, wd=wd, equilibrate=eq), H.TOL_BF16,
+                   check_stats=not eq)
+
+
+def test_fp32_step_mixed_shapes_one_shot_api(env):
+    """muon_step_batched (no plan) with fp32 grads and the fp32 Newton-Schulz path."""
+    B, torch = env
+    shapes = [(5, 9), (64, 48), (100, 300)]
+    W0 = [H.seeded(r, c, 50 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded(r, c, 60 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(3)]
+    hp = H.gpu_hp(B, mode="muongs", wd=0.05, ns_fp32=True)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.float32, use_plan=False)
+    H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs", wd=0.05), H.TOL_FP32)
+
+
+def test_muongs_invariants_on_gpu(env):
+    """<W_t, O~> = 0 and ||W_{t+1}||^2 = ||W_t||^2 + lr^2 ||O~||^2 (wd = 0), at fp32 level."""
+    B, torch = env
+    W0 = [H.seeded(96, 160, 5, 0.02)]
+    grads = [[H.seeded_bf16(96, 160, 70 + t, 1e-3)] for t in range(3)]
+    gpu = H.run_steps(B, torch, W0, grads, H.gpu_hp(B, mode="muongs"), torch.bfloat16)
+    W_prev = W0[0].astype(np.float64)
+    for t in range(3):
+        W = gpu[t][0][0]
+        O_t = (W_prev - W) / 0.02
+        assert abs(np.sum(W_prev * O_t)) <= 1e-4 * np.linalg.norm(W_prev) * np.linalg.norm(O_t)
+        lhs, rhs = np.sum(W * W), np.sum(W_prev * W_prev) + 0.02 ** 2 * np.sum(O_t * O_t)
+        assert abs(lhs - rhs) <= 1e-5 * rhs
+        W_prev = W
+
+
+def test_degenerate_step_inputs(env):
+    """Zero gradient from zero momentum: only the decay acts. Zero weight in MuonGS
+    mode: the projection is skipped. A 1x1 matrix."""
+    B, torch = env
+    W0 = [np.ones((8, 24), np.float32), np.zeros((16, 16), np.float32), np.full((1, 1), 0.5, np.float32)]
+    grads = [[np.zeros((8, 24), np.float32), H.seeded_bf16(16, 16, 9, 1e-3),
+              np.full((1, 1), -1e-3, np.float32)]]
+    hp = H.gpu_hp(B, mode="muongs", wd=0.1)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.bfloat16)
+    assert np.allclose(gpu[0][0][0], (1 - 0.02 * 0.1) * W0[0], rtol=0, atol=1e-7)
+    H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs", wd=0.1), H.TOL_BF16)

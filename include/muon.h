@@ -211,6 +211,28 @@ MUON_API muon_status_t muon_plan_profile_enable(muon_plan_t plan, int enable);
  * or -1 on a CUDA error. */
 MUON_API int muon_plan_profile_read(muon_plan_t plan, muon_profile_entry_t* out, int max_entries);
 
+/* ---- Newton-Schulz of one matrix without any caller workspace ----
+ * The pages have no counterpart of this call: it exists for callers that cannot
+ * call cudaMalloc. Examples: code that runs under a memory pool or framework
+ * allocator owning all device memory, which must not be bypassed; code that
+ * cannot afford the device-wide synchronisation cudaMalloc/cudaFree may imply.
+ * Same result as muon_newton_schulz_batched for that one matrix (X in, O out,
+ * device pointers, dtype F32 or BF16 for both). Scratch is the library's own
+ * 32 MiB static device array, which every GPU that loads the library keeps
+ * until exit. A matrix whose scratch needs exceed it is rejected with
+ * MUON_ERR_WORKSPACE before anything is enqueued. In bf16 that is 2*(m*ld_n +
+ * m*ld_m)*2 bytes plus 2 KiB, with m <= n the sorted sides and ld_* rounded up
+ * to 64, so 1024 x 4096 fits and 2048 x 2048 does not.
+ * All calls share that array: calls that overlap on the GPU (two streams or
+ * two host threads) race and must be serialised by the caller. The first call
+ * on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current), so make it before any stream capture.
+ * status_dev: optional device uint32 that receives MUON_ERR_TIMEOUT if a bounded
+ * wait inside a kernel gives up (cleared to 0 at the start of the call). */
+MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matrix_t* mat,
+                                                  const muon_hparams_t* hp, uint32_t* status_dev,
+                                                  void* stream);
+
 /* Synchronises `stream`, returns the sticky device-side error word of the
  * workspace (MUON_OK or MUON_ERR_TIMEOUT) and clears it. The word is zeroed when
  * a plan first uses a workspace and on every muon_step_batched /

@@ -90,6 +90,8 @@ def load(path: str = LIB_PATH):
         "muon_newton_schulz_batched": (c_int, [P(MuonNSMatrix), c_int, P(MuonHParams), c_void_p,
                                                c_size_t, c_void_p]),
         "muon_query_device_status": (c_int, [c_void_p, c_void_p]),
+        "muon_newton_schulz_noalloc": (c_int, [P(MuonNSMatrix), P(MuonHParams), c_void_p, c_void_p]),
+        "muon_plan_profile_enable": (c_int, [c_void_p, c_int]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -279,3 +281,19 @@ def newton_schulz(xs, outs, hp: MuonHParams, workspace=None, stream=None):
                                           workspace.numel(), _stream_ptr(stream)),
            "muon_newton_schulz_batched")
     return workspace
+
+
+def newton_schulz_noalloc(x, o, hp: MuonHParams, status=None, stream=None):
+    """O = NS(X / (||X||_F + eps)) for one matrix, using the library's static scratch
+    instead of a workspace (for callers that cannot allocate device memory).
+    status: optional CUDA int32/uint32 one-element tensor for the device error word."""
+    lib = load()
+    _check_2d(x, "X")
+    _check_2d(o, "O")
+    if x.dtype != o.dtype or tuple(x.shape) != tuple(o.shape):
+        raise MuonError(3, "X and O must have the same dtype and shape")
+    m = MuonNSMatrix(x.data_ptr(), o.data_ptr(), x.size(0), x.size(1), max(x.stride(0), x.size(1)),
+                     max(o.stride(0), o.size(1)), _dtype_code(x), 0)
+    _check(lib.muon_newton_schulz_noalloc(ctypes.byref(m), ctypes.byref(hp),
+                                          status.data_ptr() if status is not None else None,
+                                          _stream_ptr(stream)), "muon_newton_schulz_noalloc")

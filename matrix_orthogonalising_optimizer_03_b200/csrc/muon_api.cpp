@@ -543,9 +543,9 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
   const int nc = static_cast<int>(p->classes.size());
   for (int it = 0; it < hp.ns_steps; ++it) {
     for (int phase = PH_GRAM; phase <= PH_APPLY; ++phase) {
-      for (int c0 = 0; c0 < nc; c0 += kMaxClassesPerLaunch) {
+      for (int c0 = 0; p->x_fp32 && c0 < nc; c0 += kMaxClassesPerLaunch) {
         const int cn = std::min(kMaxClassesPerLaunch, nc - c0);
-        if (p->x_fp32) {
+        {
           NsPhaseArgs a{};
           a.num_classes = cn;
           a.phase = phase;
@@ -568,43 +568,63 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
           double fl = 0;
           for (int c = 0; c < cn; ++c) fl += class_phase_flops(p->classes[c0 + c], phase);
           ps.done(PK_GRAM + phase, fl, 0.0);
-        } else {
-          TcParams P;
-          std::memset(&P, 0, sizeof(P));
-          NsPhaseArgs& a = P.args;
-          a.num_classes = cn;
-          a.phase = phase;
-          a.a = hp.ns_coeffs[0];
-          a.b = hp.ns_coeffs[1];
-          a.c = hp.ns_coeffs[2];
-          a.first_iter = it == 0 ? 1 : 0;
-          a.eps = hp.eps;
-          a.scal = ea.scal;
-          a.err = ea.err;
-          int tiles = 0;
-          for (int c = 0; c < cn; ++c) {
-            const ClassMaps& cm = p->maps[c0 + c];
-            fill_class_args(p, base, c0 + c, phase, it, &a.cls[c], tc_block_m(), tc_block_n(phase),
-                            tc_block_k());
-            a.tile_base[c] = tiles;
-            tiles += a.cls[c].count * a.cls[c].tiles_per_mat;
-            if (phase == PH_GRAM) {
-              P.ta[c] = cm.x128[it % 2];
-              P.tb[c] = cm.x128[it % 2];
-            } else if (phase == PH_POLY) {
-              P.ta[c] = cm.s128;
-              P.tb[c] = cm.s128;
-            } else {
-              P.ta[c] = cm.p128;
-              P.tb[c] = cm.x64[it % 2];
+        }
+      }
+      if (!p->x_fp32) {
+        // tensor cores: classes with m a multiple of 256 run on CTA pairs (256 x 256
+        // tiles), the others on single CTAs; at most kMaxClassesPerLaunch per launch
+        for (int pair = 1; pair >= 0; --pair) {
+          std::vector<int> ids;
+          for (int c = 0; c < nc; ++c)
+            if ((p->classes[c].m % kPairTile == 0) == (pair == 1)) ids.push_back(c);
+          for (size_t g0 = 0; g0 < ids.size(); g0 += kMaxClassesPerLaunch) {
+            const int cn = static_cast<int>(std::min<size_t>(kMaxClassesPerLaunch, ids.size() - g0));
+            TcParams P;
+            std::memset(&P, 0, sizeof(P));
+            NsPhaseArgs& a = P.args;
+            a.num_classes = cn;
+            a.phase = phase;
+            a.a = hp.ns_coeffs[0];
+            a.b = hp.ns_coeffs[1];
+            a.c = hp.ns_coeffs[2];
+            a.first_iter = it == 0 ? 1 : 0;
+            a.eps = hp.eps;
+            a.scal = ea.scal;
+            a.err = ea.err;
+            int tiles = 0;
+            double fl = 0;
+            for (int c = 0; c < cn; ++c) {
+              const int cid = ids[g0 + c];
+              const ClassMaps& cm = p->maps[cid];
+              const int bm = pair ? kPairTile : tc_block_m();
+              const int bn = pair ? kPairTile : tc_block_n(phase);
+              fill_class_args(p, base, cid, phase, it, &a.cls[c], bm, bn, tc_block_k());
+              a.tile_base[c] = tiles;
+              tiles += a.cls[c].count * a.cls[c].tiles_per_mat;
+              fl += class_phase_flops(p->classes[cid], phase);
+              if (phase == PH_GRAM) {
+                P.ta[c] = cm.x128[it % 2];
+                P.tb[c] = cm.x128[it % 2];
+                P.td[c] = cm.s128;
+              } else if (phase == PH_POLY) {
+                P.ta[c] = cm.s128;
+                P.tb[c] = cm.s128;
+                P.tc[c] = cm.s128;
+                P.td[c] = cm.p128;
+              } else {
+                P.ta[c] = cm.p128;
+                P.tb[c] = cm.x64[it % 2];
+                P.tc[c] = cm.x128[it % 2];
+                P.td[c] = cm.x128[(it + 1) % 2];
+              }
             }
+            a.tile_base[cn] = tiles;
+            ProfScope ps(p, stream);
+            const cudaError_t e = pair ? launch_ns_phase_tc_pair(P, num_sms, stream)
+                                       : launch_ns_phase_tc(P, num_sms, stream);
+            if (e != cudaSuccess) return MUON_ERR_CUDA;
+            ps.done(PK_GRAM + phase, fl, 0.0);
           }
-          a.tile_base[cn] = tiles;
-          ProfScope ps(p, stream);
-          if (launch_ns_phase_tc(P, num_sms, stream) != cudaSuccess) return MUON_ERR_CUDA;
-          double fl = 0;
-          for (int c = 0; c < cn; ++c) fl += class_phase_flops(p->classes[c0 + c], phase);
-          ps.done(PK_GRAM + phase, fl, 0.0);
         }
       }
     }

@@ -52,7 +52,7 @@ struct ClassInfo {
   int64_t off_x[2], off_s, off_p;  // workspace byte offsets of the slabs
 };
 
-constexpr int kMaxClassesPerLaunch = 8;
+constexpr int kMaxClassesPerLaunch = 4;
 constexpr int kElemTileR = 32;   // elementwise tile: rows (storage frame)
 constexpr int kElemTileC = 64;   // elementwise tile: cols
 

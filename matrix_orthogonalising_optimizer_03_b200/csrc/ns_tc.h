@@ -7,12 +7,14 @@
 
 namespace muon {
 
-// Kernel parameters: per class, the tensor maps of the A and B operands of the
-// phase, plus the phase arguments. Passed as a __grid_constant__ parameter so
+// Kernel parameters: per class, the tensor maps of the A and B operands, of the
+// epilogue's C tile and of the output, plus the phase arguments. Passed as a __grid_constant__ parameter so
 // the TMA unit reads the maps from parameter space.
 struct TcParams {
-  CUtensorMap ta[kMaxClassesPerLaunch];
-  CUtensorMap tb[kMaxClassesPerLaunch];
+  CUtensorMap ta[kMaxClassesPerLaunch];  // A operand (64 x 128 boxes)
+  CUtensorMap tb[kMaxClassesPerLaunch];  // B operand
+  CUtensorMap tc[kMaxClassesPerLaunch];  // C tile of the epilogue (POLY: S, APPLY: X)
+  CUtensorMap td[kMaxClassesPerLaunch];  // output (GRAM: S, POLY: P, APPLY: X')
   NsPhaseArgs args;
 };
 
@@ -22,6 +24,11 @@ int tc_block_n(int phase);
 int tc_block_k();
 
 cudaError_t launch_ns_phase_tc(const TcParams& P, int num_sms, cudaStream_t s);
+
+// CTA-pair launch: 256 x 256 tiles (tiles_i = ceil(m/256), tiles_j = ceil(cols/256)),
+// for classes whose m is a multiple of 256. Same tensor maps as the single-CTA launch.
+cudaError_t launch_ns_phase_tc_pair(const TcParams& P, int num_sms, cudaStream_t s);
+constexpr int kPairTile = 256;
 
 bool encode_slab_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int64_t rows,
                           int64_t count, int64_t ld, int box_inner, int box_rows);

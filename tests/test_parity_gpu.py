@@ -30,7 +30,9 @@ def _ns_gpu(B, torch, xs, hp, dtype):
 
 
 SMALL = [(1, 1), (1, 40), (40, 1), (17, 33), (33, 17), (64, 64), (128, 256), (256, 128),
-         (129, 130), (200, 700), (700, 200), (320, 512), (512, 320)]
+         (129, 130), (200, 700), (700, 200), (320, 512), (512, 320),
+         # m a multiple of 256: the CTA-pair kernel (ragged n included)
+         (256, 256), (512, 700), (768, 1000), (1000, 768)]
 
 
 @pytest.mark.parametrize("coeffs,tol", [((1.0, 0.0, 0.0), 1e-2), ((0.0, 1.0, 0.0), 1e-2),
@@ -39,7 +41,8 @@ def test_tensor_core_phases_isolated(env, coeffs, tol):
     """One iteration with (a,b,c) = e1, e2, e3 isolates a*X (APPLY epilogue), S X (GRAM
     then APPLY) and S^2 X (GRAM, POLY, APPLY): each against the literal recurrence."""
     B, torch = env
-    shapes = [(17, 33), (128, 256), (129, 130), (320, 512), (512, 320), (200, 700)]
+    shapes = [(17, 33), (128, 256), (129, 130), (320, 512), (512, 320), (200, 700),
+              (256, 300), (512, 512), (768, 1000)]
     xs = [H.seeded_bf16(r, c, 10 + i, 1.0) for i, (r, c) in enumerate(shapes)]
     hp = B.hparams(ns_coeffs=coeffs, ns_steps=1)
     got = _ns_gpu(B, torch, xs, hp, torch.bfloat16)
@@ -91,7 +94,7 @@ def test_single_128x256_fp32_ten_steps(env, mode):
 
 
 STEP_SHAPES = [(17, 33), (33, 17), (128, 256), (256, 128), (200, 700), (320, 512), (512, 320),
-               (384, 384)]
+               (384, 384), (512, 700), (768, 512)]
 
 
 @pytest.mark.parametrize("mode,wd,eq", [("muongs", 0.0, False), ("muon", 0.1, False),

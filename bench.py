@@ -38,6 +38,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gpt160m")
+    ap.add_argument("--run", type=int, default=0,
+                    help="which hyper-parameter setting of the workload (e.g. gpt400m: 0 MuonGS, 1 Muon+wd)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -176,7 +178,7 @@ def run_reference(args, rank: int, world: int):
         return 0
     from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
     w = wl.WORKLOADS[args.workload]
-    run = w.runs[0]
+    run = w.runs[args.run]
     per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_sample(w, run, 0.0, rotate=i)
@@ -229,25 +231,27 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     B.load()
     w = wl.WORKLOADS[args.workload]
-    run = w.runs[0]
+    run = w.runs[args.run]
     specs = w.matrices()
     gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
     gsz = 2 if w.grad_dtype == "bf16" else 4
 
-    # resident inputs: W (fp32), M (fp32, zero), G (one flat buffer, views per matrix)
+    # resident inputs: W (fp32), M (fp32, zero), G (one flat buffer, views per matrix),
+    # drawn on the device from the shape set's distributions (seeded)
     numel = sum(s.rows * s.cols for s in specs)
+    Ws, G_src = wl.device_inputs(w, dev, seed=rank)
     g_flat = torch.empty(numel, dtype=gdt, device=dev)
-    g_host = torch.empty(numel, dtype=gdt, pin_memory=True)
-    Ws, Ms, Gs = [], [], []
+    Ms, Gs = [], []
     off = 0
-    for s in specs:
-        Ws.append(torch.from_numpy(wl.weight(w, s)).to(dev))
+    for s, g in zip(specs, G_src):
         Ms.append(torch.zeros(s.rows, s.cols, dtype=torch.float32, device=dev))
-        gv = g_host[off:off + s.rows * s.cols].view(s.rows, s.cols)
-        gv.copy_(torch.from_numpy(wl.grad(w, s, 0)).to(gdt))
-        Gs.append(g_flat[off:off + s.rows * s.cols].view(s.rows, s.cols))
+        gv = g_flat[off:off + s.rows * s.cols].view(s.rows, s.cols)
+        gv.copy_(g)
+        Gs.append(gv)
         off += s.rows * s.cols
-    g_flat.copy_(g_host)
+    del G_src
+    g_host = torch.empty(numel, dtype=gdt, pin_memory=True)
+    g_host.copy_(g_flat)
     hp = B.hparams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
                    equilibrate=run.equilibrate, ns_fp32=w.ns_fp32)
     plan = B.Plan(Ws, Gs, Ms, hp)
@@ -328,6 +332,7 @@ def main():
             "config": {"workload": w.name, "matrices": w.n_matrices, "params": w.n_params,
                        "mode": run.mode, "weight_decay": run.weight_decay,
                        "equilibrate": run.equilibrate, "ns_steps": 5, "grad_dtype": w.grad_dtype,
+                       "ns_path": "fp32 CUDA cores" if w.ns_fp32 else "bf16 tcgen05",
                        "ns_tflops_per_step": wl.workload_ns_flops(w) / 1e12,
                        "l2": "inputs larger than L2 (W+M+G = %.0f MB vs 126 MB)" % (
                            numel * (8 + gsz) / 1e6),

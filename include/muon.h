@@ -233,6 +233,13 @@ MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matrix_t* mat,
                                                   const muon_hparams_t* hp, uint32_t* status_dev,
                                                   void* stream);
 
+/* Self-test of the device-side timeout path: launches one thread that waits, with
+ * the same bounded wait the pipelined kernels use, on an mbarrier nothing arrives
+ * at, for limit_cycles SM clock cycles (1 .. 2e9), then records MUON_ERR_TIMEOUT
+ * in the workspace's error word (read it with muon_query_device_status). The
+ * workspace needs only its first 256 bytes. Nothing faults and nothing hangs. */
+MUON_API muon_status_t muon_wait_probe(void* workspace, int64_t limit_cycles, void* stream);
+
 /* Synchronises `stream`, returns the sticky device-side error word of the
  * workspace (MUON_OK or MUON_ERR_TIMEOUT) and clears it. The word is zeroed when
  * a plan first uses a workspace and on every muon_step_batched /

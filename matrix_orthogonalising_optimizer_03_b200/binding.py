@@ -92,6 +92,7 @@ def load(path: str = LIB_PATH):
         "muon_query_device_status": (c_int, [c_void_p, c_void_p]),
         "muon_newton_schulz_noalloc": (c_int, [P(MuonNSMatrix), P(MuonHParams), c_void_p, c_void_p]),
         "muon_plan_profile_enable": (c_int, [c_void_p, c_int]),
+        "muon_wait_probe": (c_int, [c_void_p, c_int64, c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

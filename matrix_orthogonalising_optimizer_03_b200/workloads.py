@@ -162,3 +162,47 @@ def normal(rows: int, cols: int, seed: int, std: float, bf16: bool = False) -> n
     g = np.random.Generator(np.random.Philox(np.random.SeedSequence([BASE_SEED, 1000, seed])))
     x = g.standard_normal((rows, cols), dtype=np.float32) * np.float32(std)
     return bf16_round(x) if bf16 else x
+
+
+def device_inputs(w: Workload, device, seed: int = 0, exact=(), step: int = 0):
+    """W_0 and G_step for every matrix of a shape set, drawn on `device` with torch's
+    seeded generator from the same distributions as `weight` / `grad`:
+    N(0, w_std^2) weights; N(0, g_std^2), g_std * Student-t(3) (a normal over the root
+    mean square of three normals), or exp(N(0,1)) row scales times N(0, g_std^2)
+    gradients, rounded to bf16 when the set's gradients are bf16. Matrices whose
+    index is in `exact` get the host generator's values instead, so that the oracle
+    can be run on them with identical inputs. Returns (Ws fp32, Gs) as lists."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(np.random.SeedSequence([BASE_SEED, w.wid, seed, step]).generate_state(1)[0]))
+    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    exact = set(exact)
+    Ws, Gs = [], []
+    for spec in w.matrices():
+        shape = (spec.rows, spec.cols)
+        if spec.index in exact:
+            Ws.append(torch.from_numpy(weight(w, spec)).to(device))
+            Gs.append(torch.from_numpy(grad(w, spec, step)).to(device=device, dtype=gdt))
+            continue
+        Ws.append(torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * w.w_std)
+        z = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+        if w.grad_dist == "student_t3":
+            v = torch.randn((3,) + shape, generator=gen, device=device, dtype=torch.float32)
+            z = z / torch.sqrt((v * v).mean(0))
+        elif w.grad_dist == "rowscaled":
+            z = z * torch.exp(torch.randn((spec.rows, 1), generator=gen, device=device))
+        Gs.append((z * w.g_std).to(gdt))
+    return Ws, Gs
+
+
+def sample_indices(w: Workload, extra: int = 3, seed: int = 7) -> List[int]:
+    """One matrix per shape class (its first) plus `extra` seeded picks: the matrices a
+    full-size parity check compares with the oracle one by one."""
+    first = {}
+    for s in w.matrices():
+        first.setdefault((s.rows, s.cols), s.index)
+    picks = sorted(first.values())
+    rng = np.random.default_rng(seed)
+    rest = [i for i in range(w.n_matrices) if i not in picks]
+    picks += sorted(rng.choice(rest, size=min(extra, len(rest)), replace=False).tolist())
+    return picks

@@ -208,6 +208,25 @@ def run_reference(args, rank: int, world: int):
     return 0
 
 
+# ------------------------------------------------------------------ multi-rank timing
+def rank_max(x: float, world: int, device="cpu") -> float:
+    """The maximum of x over all ranks of the default process group (x itself at
+    world 1). Every rank must call it at the same point."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(steps: int, world: int, ms_max: float) -> float:
+    """Whole-job shape-set steps per second: every rank steps its own copy of the
+    shape set `steps` times (weak scaling), timed by the slowest rank."""
+    return steps * world / (ms_max / 1e3)
+
+
 # ------------------------------------------------------------------ GPU arm
 def main():
     args = parse_args()
@@ -273,11 +292,7 @@ def main():
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return rank_max(x, world, dev)
 
     # 1) device-timed region: K steps, inputs resident (W+M+G far larger than L2)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -323,9 +338,8 @@ def main():
                "sample": f"float64 oracle on {n} matrices ({rounds} per shape class) of the "
                          f"{w.name} shape set, extrapolated to one full step by class counts"}
     if rank == 0:
-        steps_all = args.steps * world
         line = {
-            "metric": "muon_steps_per_s", "value": steps_all / (ms / 1e3), "unit": "steps/s",
+            "metric": "muon_steps_per_s", "value": throughput(args.steps, world, ms), "unit": "steps/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32" if w.ns_fp32 else "bf16", "data": "synthetic",
@@ -343,7 +357,7 @@ def main():
                             "ms_per_step": v["total_ms"] / args.steps} for k, v in prof.items()
                         if v["launches"]},
             "gpu_launches": int(round(launches_per_step * args.steps)),
-            "e2e": {"value": steps_all / (ms_e2e / 1e3), "unit": "steps/s",
+            "e2e": {"value": throughput(args.steps, world, ms_e2e), "unit": "steps/s",
                     "h2d_bytes_per_step": numel * gsz, "d2h_bytes_per_step": stats.numel() * 4},
             "clocks": clocks,
             "cpu_baseline": cpu,

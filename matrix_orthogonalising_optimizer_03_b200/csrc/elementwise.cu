@@ -9,9 +9,13 @@
 //                 scale (a7), GS coefficient (a8), statistics, update coefficients.
 //   post_apply    a9: W <- cw*W + co*D*O (or, Newton-Schulz only, O out).
 //
-// Work unit: a 32 x 64 tile of the matrix in its storage frame, 256 threads,
-// 8 consecutive columns per thread (128-bit accesses when aligned). The tile
-// of each block is found by binary search over a per-matrix tile prefix.
+// Work unit: a 128 x 256 super-tile of the matrix in its storage frame per
+// 256-thread block, walked as 4 x 4 sub-tiles of 32 x 64 (8 consecutive columns
+// per thread, 128-bit accesses when aligned). The super-tile of each block is
+// found by binary search over a per-matrix tile prefix. Per-matrix sums use one
+// atomic per block; the equilibration row / column sums are reduced inside the
+// block (shuffles for rows, a shared-memory transpose for columns) and use one
+// atomic per row and per column of the super-tile.
 #include <cuda_runtime.h>
 
 #include "muon_internal.h"
@@ -21,8 +25,10 @@ namespace muon {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTR = kElemTileR;  // 32 rows
-constexpr int kTC = kElemTileC;  // 64 cols
+constexpr int kTR = 32;   // sub-tile rows
+constexpr int kTC = 64;   // sub-tile cols
+constexpr int kSubR = kElemTileR / kTR;  // 4 sub-tiles down a super-tile
+constexpr int kSubC = kElemTileC / kTC;  // 4 sub-tiles across
 
 __device__ __forceinline__ void load8_f32(const float* p, bool vec, int valid, float (&v)[8]) {
   if (vec && valid == 8) {
@@ -134,6 +140,7 @@ __device__ __forceinline__ void load_o_tile(const ElemArgs& a, const DevMat& d, 
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < 8; ++e) o[e] = tile[lc + e][lr];
+    __syncthreads();  // the tile is reused by the next sub-tile
   }
 }
 
@@ -147,21 +154,12 @@ __device__ __forceinline__ int find_matrix(const ElemArgs& a, int b) {
 }
 
 // ------------------------------------------------------------------ ingest
-__global__ void __launch_bounds__(kThreads) ingest_kernel(const ElemArgs a) {
-  __shared__ float tile[kTC][kTR + 1];
-  __shared__ double red[1][kThreads / 32];
-  const int b = blockIdx.x;
-  const int k = find_matrix(a, b);
-  const DevMat d = a.mats[k];
-  const DevSlab s = a.slabs[k];
-  const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kTC - 1) / kTC;
-  const int r0 = (t / tiles_c) * kTR, c0 = (t % tiles_c) * kTC;
+__device__ __forceinline__ float ingest_subtile(const ElemArgs& a, const DevMat& d, const DevSlab& s,
+                                                int r0, int c0, float (*tile)[kTR + 1]) {
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
   const int r = r0 + lr, c = c0 + lc;
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
   const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
-
   float u[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) u[e] = 0.f;
@@ -180,24 +178,19 @@ __global__ void __launch_bounds__(kThreads) ingest_kernel(const ElemArgs a) {
       load8_f32(mp, vec, valid, m);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        m[e] = fmaf(a.mu, m[e], g[e]);                  // M_t = mu*M_{t-1} + G_t
+        m[e] = fmaf(a.mu, m[e], g[e]);                       // M_t = mu*M_{t-1} + G_t
         u[e] = a.nesterov ? fmaf(a.mu, m[e], g[e]) : m[e];  // U = G_t + mu*M_t
       }
       store8_f32(mp, vec, valid, m);
     }
   }
-  double acc[1] = {0.0};
-  {
-    float sq = 0.f;
+  float sq = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      // the slab holds U rounded to its storage type; ||U|| is taken of that value
-      const float q = a.x_fp32 ? u[e] : bf16_to_f32(f32_to_bf16(u[e]));
-      sq = fmaf(q, q, sq);
-    }
-    acc[0] = sq;
+  for (int e = 0; e < 8; ++e) {
+    // the slab holds U rounded to its storage type; ||U|| is taken of that value
+    const float q = a.x_fp32 ? u[e] : bf16_to_f32(f32_to_bf16(u[e]));
+    sq = fmaf(q, q, sq);
   }
-
   if (!(d.flags & MAT_TRANSPOSED)) {
     if (valid > 0) store8_slab(s.x0, a.x_fp32, (int64_t)r * s.ldx + c, valid, u);
   } else {
@@ -212,7 +205,26 @@ __global__ void __launch_bounds__(kThreads) ingest_kernel(const ElemArgs a) {
       for (int e = 0; e < 8; ++e) w[e] = tile[threadIdx.x >> 2][(threadIdx.x & 3) * 8 + e];
       store8_slab(s.x0, a.x_fp32, (int64_t)sr * s.ldx + sc, v2, w);
     }
+    __syncthreads();
   }
+  return sq;
+}
+
+__global__ void __launch_bounds__(kThreads, 8) ingest_kernel(const ElemArgs a) {
+  __shared__ float tile[kTC][kTR + 1];
+  __shared__ double red[1][kThreads / 32];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
+  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
+  float sq = 0.f;
+  for (int bi = 0; bi < kSubR && R0 + bi * kTR < d.rows; ++bi)
+    for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj)
+      sq += ingest_subtile(a, d, s, R0 + bi * kTR, C0 + bj * kTC, tile);
+  double acc[1] = {sq};
   block_sum<1>(acc, red);
   if (threadIdx.x == 0) atomicAdd(&a.scal[k].u2, acc[0]);
 }
@@ -223,67 +235,92 @@ __device__ __forceinline__ float slab_scale(const ElemArgs& a, int k) {
 }
 
 // ------------------------------------------------------------------ post_reduce
-__global__ void __launch_bounds__(kThreads) post_reduce_kernel(const ElemArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) post_reduce_kernel(const ElemArgs a) {
   __shared__ float tile[kTC][kTR + 1];
   __shared__ double red[3][kThreads / 32];
-  __shared__ float col_o2[kTC], col_wo[kTC];
+  __shared__ float colred[2][kTR][kTC + 1];
   const int b = blockIdx.x;
   const int k = find_matrix(a, b);
   const DevMat d = a.mats[k];
   const DevSlab s = a.slabs[k];
   const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kTC - 1) / kTC;
-  const int r0 = (t / tiles_c) * kTR, c0 = (t % tiles_c) * kTC;
+  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
+  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
-  const int r = r0 + lr, c = c0 + lc;
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
-  const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
-  if (a.equilibrate && threadIdx.x < kTC) {
-    col_o2[threadIdx.x] = 0.f;
-    col_wo[threadIdx.x] = 0.f;
-  }
-
-  float o[8];
-  load_o_tile(a, d, s, r0, c0, tile, o);
   const float xs = slab_scale(a, k);
-  float w[8];
-  if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w);
-  else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = 0.f;
-  }
   float ww = 0.f, wo = 0.f, oo = 0.f;
+  float row_o2[kSubR], row_wo[kSubR];  // this thread's share of its rows' sums
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    o[e] *= xs;
-    ww = fmaf(w[e], w[e], ww);
-    wo = fmaf(w[e], o[e], wo);
-    oo = fmaf(o[e], o[e], oo);
-  }
-  if (a.equilibrate) {
-    // per-row sums: the 8 threads of a row are consecutive lanes
-    float ro = oo, rw = wo;
+  for (int i = 0; i < kSubR; ++i) row_o2[i] = row_wo[i] = 0.f;
+
+  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
+    const int c0 = C0 + bj * kTC;
+    float col_o2[8], col_wo[8];
 #pragma unroll
-    for (int m = 4; m > 0; m >>= 1) {
-      ro += __shfl_xor_sync(0xffffffffu, ro, m);
-      rw += __shfl_xor_sync(0xffffffffu, rw, m);
-    }
-    if ((threadIdx.x & 7) == 0 && r < d.rows) {
-      atomicAdd(a.eq_o2 + s.eq_off + r, ro);
-      atomicAdd(a.eq_wo + s.eq_off + r, rw);
-    }
-    __syncthreads();
+    for (int e = 0; e < 8; ++e) col_o2[e] = col_wo[e] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      if (e < valid) {
-        atomicAdd(&col_o2[lc + e], o[e] * o[e]);
-        atomicAdd(&col_wo[lc + e], w[e] * o[e]);
+    for (int bi = 0; bi < kSubR; ++bi) {
+      const int r0 = R0 + bi * kTR;
+      if (r0 >= d.rows) break;  // uniform over the block
+      const int r = r0 + lr, c = c0 + lc;
+      const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+      float o[8];
+      load_o_tile(a, d, s, r0, c0, tile, o);
+      float w[8];
+      if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w);
+      else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float oe = e < valid ? o[e] * xs : 0.f;
+        ww = fmaf(w[e], w[e], ww);
+        wo = fmaf(w[e], oe, wo);
+        oo = fmaf(oe, oe, oo);
+        if (a.equilibrate) {
+          row_o2[bi] = fmaf(oe, oe, row_o2[bi]);
+          row_wo[bi] = fmaf(w[e], oe, row_wo[bi]);
+          col_o2[e] = fmaf(oe, oe, col_o2[e]);
+          col_wo[e] = fmaf(w[e], oe, col_wo[e]);
+        }
       }
     }
-    __syncthreads();
-    if (threadIdx.x < kTC && c0 + (int)threadIdx.x < d.cols) {
-      atomicAdd(a.eq_o2 + s.eq_off + d.rows + c0 + threadIdx.x, col_o2[threadIdx.x]);
-      atomicAdd(a.eq_wo + s.eq_off + d.rows + c0 + threadIdx.x, col_wo[threadIdx.x]);
+    if (a.equilibrate) {
+      // column sums over the super-tile's rows: transpose through shared memory
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        colred[0][lr][lc + e] = col_o2[e];
+        colred[1][lr][lc + e] = col_wo[e];
+      }
+      __syncthreads();
+      if (threadIdx.x < 2 * kTC) {
+        const int which = threadIdx.x / kTC, cc = threadIdx.x % kTC;
+        float sum = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < kTR; ++i) sum += colred[which][i][cc];
+        if (c0 + cc < d.cols)
+          atomicAdd((which ? a.eq_wo : a.eq_o2) + s.eq_off + d.rows + c0 + cc, sum);
+      }
+      __syncthreads();
+    }
+  }
+  if (a.equilibrate) {
+    // row sums: the 8 threads of a row are consecutive lanes
+#pragma unroll
+    for (int bi = 0; bi < kSubR; ++bi) {
+      float ro = row_o2[bi], rw = row_wo[bi];
+#pragma unroll
+      for (int m = 4; m > 0; m >>= 1) {
+        ro += __shfl_xor_sync(0xffffffffu, ro, m);
+        rw += __shfl_xor_sync(0xffffffffu, rw, m);
+      }
+      const int r = R0 + bi * kTR + lr;
+      if ((threadIdx.x & 7) == 0 && r < d.rows) {
+        atomicAdd(a.eq_o2 + s.eq_off + r, ro);
+        atomicAdd(a.eq_wo + s.eq_off + r, rw);
+      }
     }
   }
   double acc[3] = {ww, wo, oo};
@@ -382,45 +419,50 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
 }
 
 // ------------------------------------------------------------------ post_apply
-__global__ void __launch_bounds__(kThreads) post_apply_kernel(const ElemArgs a) {
+__global__ void __launch_bounds__(kThreads, 6) post_apply_kernel(const ElemArgs a) {
   __shared__ float tile[kTC][kTR + 1];
   const int b = blockIdx.x;
   const int k = find_matrix(a, b);
   const DevMat d = a.mats[k];
   const DevSlab s = a.slabs[k];
   const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kTC - 1) / kTC;
-  const int r0 = (t / tiles_c) * kTR, c0 = (t % tiles_c) * kTC;
+  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
+  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
-  const int r = r0 + lr, c = c0 + lc;
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
-  const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
-
-  float o[8];
-  load_o_tile(a, d, s, r0, c0, tile, o);
-  if (valid <= 0) return;
   const float xs = slab_scale(a, k);
-  if (a.ns_only) {
+  MatCoef cf;
+  if (!a.ns_only) cf = a.coef[k];
+  for (int bi = 0; bi < kSubR && R0 + bi * kTR < d.rows; ++bi) {
+    for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
+      const int r0 = R0 + bi * kTR, c0 = C0 + bj * kTC;
+      const int r = r0 + lr, c = c0 + lc;
+      const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+      float o[8];
+      load_o_tile(a, d, s, r0, c0, tile, o);
+      if (valid <= 0) continue;
+      if (a.ns_only) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) o[e] *= xs;
-    if (d.flags & MAT_G_BF16)
-      store8_bf16(reinterpret_cast<uint16_t*>(d.W) + (int64_t)r * d.ld_w + c, vec, valid, o);
-    else
-      store8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, o);
-    return;
-  }
-  const MatCoef cf = a.coef[k];
-  float w[8];
-  float* wp = d.W + (int64_t)r * d.ld_w + c;
-  load8_f32(wp, vec, valid, w);
-  const float rowf = cf.axis == 1 ? a.eq_o2[s.eq_off + r] : 1.f;
+        for (int e = 0; e < 8; ++e) o[e] *= xs;
+        if (d.flags & MAT_G_BF16)
+          store8_bf16(reinterpret_cast<uint16_t*>(d.W) + (int64_t)r * d.ld_w + c, vec, valid, o);
+        else
+          store8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, o);
+        continue;
+      }
+      float w[8];
+      float* wp = d.W + (int64_t)r * d.ld_w + c;
+      load8_f32(wp, vec, valid, w);
+      const float rowf = cf.axis == 1 ? a.eq_o2[s.eq_off + r] : 1.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    float f = xs * rowf;
-    if (cf.axis == 2 && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
-    w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
+      for (int e = 0; e < 8; ++e) {
+        float f = xs * rowf;
+        if (cf.axis == 2 && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+        w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
+      }
+      store8_f32(wp, vec, valid, w);
+    }
   }
-  store8_f32(wp, vec, valid, w);
 }
 
 }  // namespace

@@ -32,10 +32,12 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t round_up64(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct ClassMaps {
-  CUtensorMap x128[2];  // X slabs, 64 x 128 boxes (K-major operand)
+  CUtensorMap x128[2];  // X slabs, 64 x 128 boxes (K-major operand, output)
   CUtensorMap x64[2];   // X slabs, 64 x 64 boxes (MN-major operand of APPLY)
-  CUtensorMap s128;     // S slab
-  CUtensorMap p128;     // P slab
+  CUtensorMap s128;     // S slab, 64 x 128 boxes
+  CUtensorMap s64;      // S slab, 64 x 64 boxes (mirror blocks below the diagonal)
+  CUtensorMap p128;     // P' slab, 64 x 128 boxes
+  CUtensorMap p64;      // P' slab, 64 x 64 boxes
 };
 
 }  // namespace
@@ -378,7 +380,9 @@ muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t str
         ok = ok && encode_slab_map_bf16(&cm.x64[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 64);
       }
       ok = ok && encode_slab_map_bf16(&cm.s128, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 128);
+      ok = ok && encode_slab_map_bf16(&cm.s64, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 64);
       ok = ok && encode_slab_map_bf16(&cm.p128, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 128);
+      ok = ok && encode_slab_map_bf16(&cm.p64, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 64);
       if (!ok) return MUON_ERR_CUDA;
     }
   }
@@ -602,18 +606,23 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
               a.tile_base[c] = tiles;
               tiles += a.cls[c].count * a.cls[c].tiles_per_mat;
               fl += class_phase_flops(p->classes[cid], phase);
+              // S and P' hold only their blocks on or above the (tile) diagonal; the
+              // *_t maps fetch mirror blocks for the operands below it
               if (phase == PH_GRAM) {
-                P.ta[c] = cm.x128[it % 2];
-                P.tb[c] = cm.x128[it % 2];
-                P.td[c] = cm.s128;
+                P.ta[c] = P.ta_t[c] = cm.x128[it % 2];
+                P.tb[c] = P.tb_t[c] = cm.x128[it % 2];
+                P.tc[c] = P.td[c] = cm.s128;
               } else if (phase == PH_POLY) {
                 P.ta[c] = cm.s128;
+                P.ta_t[c] = cm.s64;
                 P.tb[c] = cm.s128;
+                P.tb_t[c] = cm.s64;
                 P.tc[c] = cm.s128;
                 P.td[c] = cm.p128;
               } else {
                 P.ta[c] = cm.p128;
-                P.tb[c] = cm.x64[it % 2];
+                P.ta_t[c] = cm.p64;
+                P.tb[c] = P.tb_t[c] = cm.x64[it % 2];
                 P.tc[c] = cm.x128[it % 2];
                 P.td[c] = cm.x128[(it + 1) % 2];
               }

@@ -53,8 +53,8 @@ struct ClassInfo {
 };
 
 constexpr int kMaxClassesPerLaunch = 4;
-constexpr int kElemTileR = 32;   // elementwise tile: rows (storage frame)
-constexpr int kElemTileC = 64;   // elementwise tile: cols
+constexpr int kElemTileR = 128;  // elementwise super-tile: rows (storage frame)
+constexpr int kElemTileC = 256;  // elementwise super-tile: cols
 
 // Workspace header: the sticky device error word and a step counter.
 struct WsHeader {

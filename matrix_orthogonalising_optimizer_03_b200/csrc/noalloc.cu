@@ -227,20 +227,25 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
       }
       const void* x_in = k.x_in;
       bool ok = true;
+      // S and P' hold only their blocks on or above the diagonal; *_t maps fetch mirrors
       if (phase == PH_GRAM) {
         ok = encode_slab_map_bf16(&P.ta[0], x_in, n, m, 1, ldx, 64, 128) &&
              encode_slab_map_bf16(&P.td[0], k.s, m, m, 1, lds, 64, 128);
-        P.tb[0] = P.ta[0];
+        P.ta_t[0] = P.tb[0] = P.tb_t[0] = P.ta[0];
+        P.tc[0] = P.td[0];
       } else if (phase == PH_POLY) {
         ok = encode_slab_map_bf16(&P.ta[0], k.s, m, m, 1, lds, 64, 128) &&
+             encode_slab_map_bf16(&P.ta_t[0], k.s, m, m, 1, lds, 64, 64) &&
              encode_slab_map_bf16(&P.td[0], k.p, m, m, 1, lds, 64, 128);
-        P.tb[0] = P.ta[0];
-        P.tc[0] = P.ta[0];
+        P.tb[0] = P.tc[0] = P.ta[0];
+        P.tb_t[0] = P.ta_t[0];
       } else {
         ok = encode_slab_map_bf16(&P.ta[0], k.p, m, m, 1, lds, 64, 128) &&
+             encode_slab_map_bf16(&P.ta_t[0], k.p, m, m, 1, lds, 64, 64) &&
              encode_slab_map_bf16(&P.tb[0], x_in, n, m, 1, ldx, 64, 64) &&
              encode_slab_map_bf16(&P.tc[0], x_in, n, m, 1, ldx, 64, 128) &&
              encode_slab_map_bf16(&P.td[0], k.x_out, n, m, 1, ldx, 64, 128);
+        P.tb_t[0] = P.tb[0];
       }
       if (!ok) return MUON_ERR_CUDA;
       if (launch_ns_phase_tc(P, num_sms, s) != cudaSuccess) return MUON_ERR_CUDA;

@@ -6,27 +6,42 @@
 // TRAINING" review) as three grouped GEMM launches over every matrix of every
 // shape class in the call:
 //   GRAM   S  = alpha * X X^T            A = X (K-major), B = X (K-major), K = n
-//   POLY   P' = a*I + b*S + c * S S      A = S (K-major), B = S (K-major, S = S^T), K = m
-//   APPLY  X' = gamma * P' X             A = P' (K-major), B = X (MN-major), K = m
-// The a*X term of the recurrence is folded into P' (a*X + P X = (a I + P) X), so
-// the apply epilogue needs no second read of X; P' is rounded to bf16 once, with
-// its diagonal a + P_ii (about 0.7) in place of P_ii (about -2.7).
-// GRAM and POLY have symmetric outputs: only tiles with ti <= tj are computed and
-// each off-diagonal tile is stored twice (direct and mirrored).
-// alpha = 1/(||U||+eps)^2, gamma = 1/(||U||+eps) on the first iteration (the
-// slab holds the unnormalised U), 1 afterwards. X, S, P are stored in bf16,
+//   POLY   P' = a*I + b*S + c * S S      A = S, B = S (S = S^T), K = m
+//   APPLY  X' = gamma * P' X             A = P', B = X (MN-major), K = m
+// alpha = 1/(||U||+eps)^2 and gamma = 1/(||U||+eps) on the first iteration (the
+// slab then holds the unnormalised U), 1 afterwards. X, S, P' are stored in bf16,
 // accumulation is fp32 in TMEM.
 //
-// Kernel structure (persistent, one CTA per SM, 192 threads):
-//   warp 0   TMA producer: 128 x 64 A box and the B boxes into a STAGES-deep
-//            ring of 128B-swizzled shared-memory stages (no multicast).
-//   warp 1   TMEM allocator and MMA issuer: tcgen05.mma.cta_group::1.kind::f16,
-//            M=128, N=BN, K=16 per instruction, into one of two TMEM accumulators.
-//   warps 2-5 epilogue: tcgen05.ld 32 lanes x 32 columns, fused scale / axpy with
-//            the bf16 C operand, bf16 stores (and mirrored stores).
-// Slabs are [count][rows][ld] bf16 and are addressed by 3-D tensor maps
-// (inner dim, rows, matrix), so out-of-range rows and columns of a matrix are
-// zero-filled by TMA and never spill into the next matrix.
+// The a*X term of the recurrence is folded into P' (a*X + P X = (a I + P) X), so the
+// apply epilogue reads nothing but the accumulator; P' is rounded to bf16 once, with
+// its diagonal a + P_ii (about 0.7) in place of P_ii (about -2.7).
+//
+// Symmetric storage: S and P' are symmetric, so only their 128 x 128 blocks on or
+// above the block diagonal are computed and stored. A consumer that needs a block
+// below the diagonal (rows in block i, columns in block k < i) loads its mirror
+// block (k, i) with 64 x 64 TMA boxes and hands it to tcgen05.mma as an MN-major
+// operand (the transpose is free in the instruction descriptor).
+//
+// Kernel structure (persistent, one CTA per SM, 320 threads):
+//   warp 0     TMA producer: a STAGES-deep ring of 128B-swizzled shared-memory
+//              stages (no multicast in any form).
+//   warp 1     TMEM allocator and MMA issuer (one thread), double-buffered fp32
+//              accumulator in TMEM.
+//   warps 2-9  epilogue: two warps per TMEM lane quarter, each taking half of the
+//              columns; tcgen05.ld, fused scale / axpy, bf16 tile staged in swizzled
+//              shared memory and written with TMA bulk stores (which clip ragged
+//              edges). POLY's C tile (S) arrives by TMA one tile ahead.
+// Two variants:
+//   single CTA   tile 128 x BN (BN = 128 for GRAM / POLY, 256 for APPLY),
+//                tcgen05.mma.cta_group::1, M = 128.
+//   CTA pair     cluster of two CTAs, tile 256 x 256, tcgen05.mma.cta_group::2
+//                (M = N = 256): each CTA loads its 128 rows of A and half of B into
+//                its own shared memory (plain TMA loads whose bytes count on the first
+//                CTA's barrier) and owns 128 accumulator rows in its TMEM. Per CTA this
+//                halves the operand bytes per flop. Used for classes with m % 256 == 0.
+// Slabs are [count][rows][ld] bf16 addressed by 3-D tensor maps (inner dim, rows,
+// matrix), so out-of-range rows and columns of a matrix are zero-filled by TMA and
+// never spill into the next matrix. Every wait is bounded (see ptx.cuh).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -39,25 +54,33 @@ namespace muon {
 namespace {
 
 constexpr int BM = 128, BK = 64;
-constexpr int kEpiWarps = 4;
-constexpr int kThreadsTc = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreadsTc = 64 + 32 * kEpiWarps;  // 320
 
-template <int BN, int PHASE>
+template <int BN, int PHASE, bool PAIR>
 struct TcCfg {
-  static constexpr bool kHasC = PHASE == PH_POLY;       // epilogue reads a C tile (S)
-  static constexpr bool kSym = PHASE != PH_APPLY;       // mirrored (transposed) store
+  static constexpr bool kSym = PHASE != PH_APPLY;         // symmetric (upper-block) output
+  static constexpr bool kHasC = PHASE == PH_POLY;         // epilogue reads a C tile (S)
+  static constexpr int kNCol = PAIR ? 256 : BN;            // accumulator columns per CTA
+  static constexpr int kBRows = PAIR ? 128 : BN;           // B rows (or columns) per CTA
   static constexpr int kABytes = BM * BK * 2;
-  static constexpr int kBBytes = BN * BK * 2;
+  static constexpr int kBBytes = kBRows * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = BN == 256 ? 3 : 4;
-  static constexpr int kTileBytes = BM * BN * 2;        // one bf16 output tile (C / D staging)
-  static constexpr int kTBytes = kSym ? BN * BM * 2 : 0;  // transposed staging
-  static constexpr int kOffD = kStages * kStageBytes;
-  static constexpr int kOffT = kOffD + kTileBytes;
-  static constexpr int kOffBar = kOffT + kTBytes;
-  static constexpr int kTmemCols = 2 * BN;
-  static constexpr int kBarBytes = 256;
-  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
+  static constexpr int kStagingBytes = kHasC ? BM * kNCol * 2 : BM * 128 * 2;
+  static constexpr int kBudget = 224 * 1024;
+  static constexpr int kFit = (kBudget - kStagingBytes) / kStageBytes;
+  static constexpr int kStages = kFit > 8 ? 8 : kFit;
+  static constexpr int kOffStg = kStages * kStageBytes;
+  static constexpr int kOffBar = kOffStg + kStagingBytes;
+  static constexpr int kTmemCols = 2 * kNCol;
+  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
+  static constexpr int kMmaM = PAIR ? 256 : 128;
+  static constexpr int kMmaN = PAIR ? 256 : BN;
+  static constexpr int kTileM = PAIR ? 256 : 128;          // output tile (cluster) rows
+  static constexpr int kTileN = PAIR ? 256 : BN;           // output tile columns
+  static constexpr int kChunks = kNCol / 32;               // 32-column TMEM chunks per CTA
+  static constexpr int kRounds = kNCol / 128;              // 128-column store rounds
+  static_assert(kStages >= 3, "pipeline too shallow");
 };
 
 struct TileJob {
@@ -88,27 +111,61 @@ __device__ __forceinline__ TileJob decode(const NsPhaseArgs& p, int t, bool sym)
   return j;
 }
 
-// Byte offset of element (r, c) of a tile staged as 64-column boxes of 128 rows
-// with the 128-byte swizzle (the layout TMA reads and writes for a 64 x 128 box).
+// Byte offset of element (r, c) of a 128-row tile staged as 64-column boxes with
+// the 128-byte swizzle (the layout TMA reads and writes for a 64 x 128 box).
 __device__ __forceinline__ uint32_t sw128_off(int r, int c) {
   return static_cast<uint32_t>((c >> 6) * (BM * 128) + r * 128 +
                                ((((c >> 3) & 7) ^ (r & 7)) << 4) + ((c & 7) << 1));
 }
 
-template <int BN, int PHASE>
+// Whether k-block kb of the operand rows of a tile starting at row tile_row0 lies
+// below the stored block diagonal (block size G) and must be read from its mirror.
+// G is the class's tile height: 128 for single-CTA classes, 256 for CTA-pair
+// classes (whose diagonal 256 x 256 tiles are stored whole, so that both CTAs of a
+// pair always agree on the layout of a k-block).
+__device__ __forceinline__ bool below_diag(bool sym_operand, int tile_row0, int kb, int G) {
+  return sym_operand && (kb * BK) / G < tile_row0 / G;
+}
+
+// Loads the 128 x 64 block of a K-major operand, or its mirror as two 64 x 64
+// boxes (MN-major layout, 8 KB apart) when it lies below the diagonal.
+template <bool PAIR>
+__device__ __forceinline__ void load_k_block(uint8_t* dst, const CUtensorMap* mk,
+                                             const CUtensorMap* mt, uint64_t* bar, int row0,
+                                             int kb, int mat, bool mirrored) {
+  if (!mirrored) {
+    if (PAIR) tma_load_3d_pair(dst, mk, bar, kb * BK, row0, mat);
+    else tma_load_3d(dst, mk, bar, kb * BK, row0, mat);
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (PAIR) tma_load_3d_pair(dst + h * (64 * BK * 2), mt, bar, row0 + h * 64, kb * BK, mat);
+      else tma_load_3d(dst + h * (64 * BK * 2), mt, bar, row0 + h * 64, kb * BK, mat);
+    }
+  }
+}
+
+// Descriptor of the kk-th K = 16 slice of a staged operand block.
+__device__ __forceinline__ uint64_t op_desc(uint32_t base, int kk, bool mn_major) {
+  return mn_major ? smem_desc_sw128(base + kk * 2048, 64 * BK * 2, 1024)
+                  : smem_desc_sw128(base + kk * 32, 16, 1024);
+}
+
+template <int BN, int PHASE, bool PAIR>
 __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_constant__ TcParams P) {
-  using C = TcCfg<BN, PHASE>;
+  using C = TcCfg<BN, PHASE, PAIR>;
   constexpr bool SYM = C::kSym;
   constexpr bool HAS_C = C::kHasC;
-  constexpr bool B_MN = PHASE == PH_APPLY;
   constexpr int S = C::kStages;
-  static_assert(!SYM || BN == BM, "symmetric phases use square tiles");
+  constexpr bool A_SYM = PHASE != PH_GRAM;   // A is S (POLY) or P' (APPLY): upper blocks only
+  constexpr bool B_SYM = PHASE == PH_POLY;   // B is S
+  constexpr bool B_MN = PHASE == PH_APPLY;   // B is X read along its rows
+  static_assert(PAIR || !SYM || BN == BM, "single-CTA symmetric phases use square tiles");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* dtile = smem + C::kOffD;   // C tile in, D tile out (in place)
-  uint8_t* ttile = smem + C::kOffT;   // transposed D (symmetric phases)
+  uint8_t* stg = smem + C::kOffStg;  // output staging (POLY: the C tile, overwritten by D)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
@@ -121,6 +178,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
   const NsPhaseArgs& p = P.args;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total = p.tile_base[p.num_classes];
+  const int rank = PAIR ? static_cast<int>(cluster_cta_rank()) : 0;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nunits = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -129,7 +189,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], kEpiWarps);
+      mbar_init(&tempty[b], (PAIR ? 2 : 1) * kEpiWarps);
     }
     mbar_init(done, 1);
     mbar_init(cfull, 1);
@@ -137,11 +197,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(tmem_slot, C::kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_slot, C::kTmemCols);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -154,9 +220,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
       }
       long long q = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = unit; t < total && ok; t += nunits) {
         const TileJob j = decode(p, t, SYM);
         const int kb_n = p.cls[j.c].k_blocks;
+        const int a_row0 = j.ti * C::kTileM + rank * 128;
+        const int b_row0 = j.tj * C::kTileN + rank * (PAIR ? 128 : 0);
         for (int kb = 0; kb < kb_n; ++kb) {
           const int s = static_cast<int>(q % S);
           const uint32_t par = static_cast<uint32_t>((q / S) & 1);
@@ -166,319 +234,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           }
           uint8_t* sa = smem + s * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
-          mbar_expect_tx(&full[s], C::kStageBytes);
-          tma_load_3d(sa, &P.ta[j.c], &full[s], kb * BK, j.ti * BM, j.mat);
+          if (!PAIR || rank == 0) mbar_expect_tx(&full[s], (PAIR ? 2 : 1) * C::kStageBytes);
+          load_k_block<PAIR>(sa, &P.ta[j.c], &P.ta_t[j.c], &full[s], a_row0, kb, j.mat,
+                             below_diag(A_SYM, j.ti * C::kTileM, kb, C::kTileM));
           if (!B_MN) {
-            tma_load_3d(sb, &P.tb[j.c], &full[s], kb * BK, j.tj * BN, j.mat);
+            load_k_block<PAIR>(sb, &P.tb[j.c], &P.tb_t[j.c], &full[s], b_row0, kb, j.mat,
+                               below_diag(B_SYM, j.tj * C::kTileN, kb, C::kTileN));
           } else {
 #pragma unroll
-            for (int h = 0; h < BN / 64; ++h)
-              tma_load_3d(sb + h * (64 * BK * 2), &P.tb[j.c], &full[s], j.tj * BN + h * 64,
-                          kb * BK, j.mat);
-          }
-          ++q;
-        }
-      }
-      if (!ok) {
-        set_error(p.err, MUON_ERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      // Never leave the CTA with bulk copies still landing in its shared memory.
-      for (long long r = (q > S ? q - S : 0); r < q; ++r)
-        mbar_wait(&full[r % S], static_cast<uint32_t>((r / S) & 1), nullptr);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, B_MN);
-      long long q = 0;
-      int it = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-        const TileJob j = decode(p, t, SYM);
-        const int kb_n = p.cls[j.c].k_blocks;
-        const int ab = it & 1;
-        const uint32_t apar = static_cast<uint32_t>((it >> 1) & 1);
-        if (!mbar_wait(&tempty[ab], apar ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * BN);
-        for (int kb = 0; kb < kb_n; ++kb) {
-          const int s = static_cast<int>(q % S);
-          const uint32_t par = static_cast<uint32_t>((q / S) & 1);
-          if (!mbar_wait(&full[s], par, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
-          const uint32_t sb = sa + C::kABytes;
-#pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 64 * BK * 2, 1024)
-                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
-            umma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(&empty[s]);  // frees the stage once these MMAs have read it
-          ++q;
-        }
-        if (!ok) break;
-        umma_commit(&tfull[ab]);  // accumulator ready for the epilogue
-      }
-      if (!ok) {
-        set_error(p.err, MUON_ERR_TIMEOUT);
-        *abort_flag = 1;
-      }
-      umma_commit(done);  // arrives once every MMA issued above has completed
-      mbar_wait(done, 0, nullptr);
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue (warps 2-5)
-    const int quad = warp & 3;  // the TMEM lane quarter this warp may access
-    const int r = quad * 32 + lane;  // tile row of this thread
-    const bool leader = warp == 2 && lane == 0;
-    bool c_pending = false;
-    if (HAS_C && leader && static_cast<int>(blockIdx.x) < total) {
-      const TileJob j = decode(p, blockIdx.x, SYM);
-      mbar_expect_tx(cfull, C::kTileBytes);
-#pragma unroll
-      for (int h = 0; h < BN / 64; ++h)
-        tma_load_3d(dtile + h * (BM * 128), &P.tc[j.c], cfull, j.tj * BN + h * 64, j.ti * BM, j.mat);
-      c_pending = true;
-    }
-    // All four epilogue warps walk the same tiles and execute every named barrier,
-    // also after a failed wait (they then skip the work), so no warp can be left
-    // waiting at a barrier.
-    int it = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
-      const TileJob j = decode(p, t, SYM);
-      const NsClassArgs& k = p.cls[j.c];
-      const int ab = it & 1;
-      const uint32_t apar = static_cast<uint32_t>((it >> 1) & 1);
-      bool okw = ok && __all_sync(0xffffffffu, mbar_wait(&tfull[ab], apar, abort_flag));
-      if (okw && HAS_C) okw = __all_sync(0xffffffffu, mbar_wait(cfull, it & 1, abort_flag));
-      if (!okw && ok) {
-        ok = false;
-        if (lane == 0) {
-          set_error(p.err, MUON_ERR_TIMEOUT);
-          *abort_flag = 1;
-        }
-      }
-      const bool mirror = SYM && j.ti != j.tj;
-      if (ok) {
-        if (leader) c_pending = false;
-        tc_fence_after();
-        float scale = 1.f;
-        if (PHASE != PH_POLY && p.first_iter) {
-          const double inv = 1.0 / (sqrt(p.scal[k.first + j.mat].u2) + (double)p.eps);
-          scale = static_cast<float>(PHASE == PH_GRAM ? inv * inv : inv);
-        }
-#pragma unroll 1
-        for (int ch = 0; ch < BN / 32; ++ch) {
-          uint32_t v[32];
-          tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                        static_cast<uint32_t>(ab * BN + ch * 32),
-                    v);
-          tmem_wait_ld();
-          uint32_t packed[16];
-          // the element of this row on the global diagonal, as a column of this chunk
-          const int dcol = (j.ti * BM + r) - (j.tj * BN + ch * 32);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            const uint32_t off = sw128_off(r, ch * 32 + q4 * 8);
-            uint4 cw = make_uint4(0, 0, 0, 0);
-            if (HAS_C) cw = *reinterpret_cast<const uint4*>(dtile + off);
-            const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int i0 = q4 * 8 + 2 * e;
-              float a0 = __uint_as_float(v[i0]), a1 = __uint_as_float(v[i0 + 1]);
-              if (PHASE == PH_POLY) {
-                a0 = fmaf(p.b, __uint_as_float(cwv[e] << 16), p.c * a0);
-                a1 = fmaf(p.b, __uint_as_float(cwv[e] & 0xFFFF0000u), p.c * a1);
-                if (i0 == dcol) a0 += p.a;
-                if (i0 + 1 == dcol) a1 += p.a;
-              } else {
-                a0 *= scale;
-                a1 *= scale;
-              }
-              packed[q4 * 4 + e] = pack_bf16x2(a0, a1);
+            for (int h = 0; h < C::kBRows / 64; ++h) {
+              if (PAIR) tma_load_3d_pair(sb + h * (64 * BK * 2), &P.tb[j.c], &full[s], b_row0 + h * 64, kb * BK, j.mat);
+              else tma_load_3d(sb + h * (64 * BK * 2), &P.tb[j.c], &full[s], b_row0 + h * 64, kb * BK, j.mat);
             }
-            *reinterpret_cast<uint4*>(dtile + off) = make_uint4(
-                packed[q4 * 4], packed[q4 * 4 + 1], packed[q4 * 4 + 2], packed[q4 * 4 + 3]);
-          }
-          if (mirror) {
-            // element (r, c) of D is element (c, r) of the mirrored tile
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              *reinterpret_cast<uint16_t*>(ttile + sw128_off(ch * 32 + e, r)) =
-                  static_cast<uint16_t>(packed[e >> 1] >> ((e & 1) * 16));
-          }
-        }
-        // the accumulator may be reused as soon as it has been read
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[ab]);
-        fence_proxy_async_smem();
-      }
-      named_barrier(1, kEpiWarps * 32);
-      if (leader && ok) {
-        // boxes that start beyond the matrix edge hold nothing to store
-        const int ncols = PHASE == PH_APPLY ? k.n : k.m;
-#pragma unroll
-        for (int h = 0; h < BN / 64; ++h)
-          if (j.tj * BN + h * 64 < ncols)
-            tma_store_3d(&P.td[j.c], dtile + h * (BM * 128), j.tj * BN + h * 64, j.ti * BM, j.mat);
-        if (mirror) {
-#pragma unroll
-          for (int h = 0; h < BM / 64; ++h)
-            if (j.ti * BM + h * 64 < k.m)
-              tma_store_3d(&P.td[j.c], ttile + h * (BM * 128), j.ti * BM + h * 64, j.tj * BN, j.mat);
-        }
-        tma_store_commit();
-        tma_store_wait_read();  // staging buffers are free again
-        const int tn = t + static_cast<int>(gridDim.x);
-        if (HAS_C && tn < total) {
-          const TileJob jn = decode(p, tn, SYM);
-          mbar_expect_tx(cfull, C::kTileBytes);
-#pragma unroll
-          for (int h = 0; h < BN / 64; ++h)
-            tma_load_3d(dtile + h * (BM * 128), &P.tc[jn.c], cfull, jn.tj * BN + h * 64,
-                        jn.ti * BM, jn.mat);
-          c_pending = true;
-        }
-      }
-      named_barrier(1, kEpiWarps * 32);
-    }
-    if (leader) {
-      tma_store_wait_all();
-      if (c_pending) mbar_wait(cfull, it & 1, nullptr);  // a C tile still landing
-    }
-  }
-
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, C::kTmemCols);
-  }
-}
-
-// ============================================================================
-// CTA-pair variant: a cluster of two CTAs computes a 256 x 256 tile with
-// tcgen05.mma.cta_group::2 (M = 256, N = 256). CTA r of the pair loads rows
-// [128r, 128r+128) of the A tile and half r of the B tile into its own shared
-// memory (plain TMA loads whose bytes are counted on the first CTA's barrier),
-// and owns rows [128r, 128r+128) of the accumulator in its TMEM. Per CTA this
-// halves the operand bytes per flop of the 128 x 256 single-CTA tile.
-// Symmetric phases: tile (ti, tj), tj >= ti, in 256-blocks; each CTA's two
-// 128 x 128 sub-blocks (si = 2ti + r, sj = 2tj + h) are stored directly when
-// sj >= si and also mirrored when sj > si (sub-blocks below the diagonal come
-// from the mirror of another sub-block).
-template <int PHASE>
-struct PairCfg {
-  static constexpr int kABytes = 128 * BK * 2;
-  static constexpr int kBBytes = 128 * BK * 2;
-  static constexpr int kStageBytes = kABytes + kBBytes;  // 32 KB per CTA
-  static constexpr int kStages = PHASE == PH_APPLY ? 5 : 4;
-  static constexpr int kCDBytes = 128 * 256 * 2;          // C tile in, D tile out
-  static constexpr int kTBytes = PHASE == PH_APPLY ? 0 : 128 * 128 * 2;  // transposed sub-block
-  static constexpr int kOffCD = kStages * kStageBytes;
-  static constexpr int kOffT = kOffCD + kCDBytes;
-  static constexpr int kOffBar = kOffT + kTBytes;
-  static constexpr int kTmemCols = 512;                   // two 256-column accumulators
-  static constexpr int kSmemBytes = kOffBar + 256 + 1024;
-};
-
-template <int PHASE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
-    ns_tc_pair_kernel(const __grid_constant__ TcParams P) {
-  using C = PairCfg<PHASE>;
-  constexpr bool SYM = PHASE != PH_APPLY;
-  constexpr bool HAS_C = PHASE == PH_POLY;
-  constexpr bool B_MN = PHASE == PH_APPLY;
-  constexpr int S = C::kStages;
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint8_t* cd = smem + C::kOffCD;
-  uint8_t* tt = smem + C::kOffT;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* empty = full + S;
-  uint64_t* tfull = empty + S;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
-  uint64_t* cfull = done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cfull + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const NsPhaseArgs& p = P.args;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int total = p.tile_base[p.num_classes];
-  const uint32_t rank = cluster_cta_rank();
-  const int cluster_id = static_cast<int>(blockIdx.x >> 1);
-  const int nclusters = static_cast<int>(gridDim.x >> 1);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 2 * kEpiWarps);
-    }
-    mbar_init(done, 1);
-    mbar_init(cfull, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, C::kTmemCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      for (int c = 0; c < p.num_classes; ++c) {
-        tma_prefetch(&P.ta[c]);
-        tma_prefetch(&P.tb[c]);
-      }
-      long long q = 0;
-      bool ok = true;
-      for (int t = cluster_id; t < total && ok; t += nclusters) {
-        const TileJob j = decode(p, t, SYM);
-        const int kb_n = p.cls[j.c].k_blocks;
-        for (int kb = 0; kb < kb_n; ++kb) {
-          const int s = static_cast<int>(q % S);
-          const uint32_t par = static_cast<uint32_t>((q / S) & 1);
-          if (!mbar_wait(&empty[s], par ^ 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = smem + s * C::kStageBytes;
-          uint8_t* sb = sa + C::kABytes;
-          if (rank == 0) mbar_expect_tx(&full[s], 2 * C::kStageBytes);
-          tma_load_3d_pair(sa, &P.ta[j.c], &full[s], kb * BK, j.ti * 256 + static_cast<int>(rank) * 128,
-                           j.mat);
-          if (!B_MN) {
-            tma_load_3d_pair(sb, &P.tb[j.c], &full[s], kb * BK,
-                             j.tj * 256 + static_cast<int>(rank) * 128, j.mat);
-          } else {
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tma_load_3d_pair(sb + h * (64 * BK * 2), &P.tb[j.c], &full[s],
-                               j.tj * 256 + static_cast<int>(rank) * 128 + h * 64, kb * BK, j.mat);
           }
           ++q;
         }
@@ -487,22 +254,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
         set_error(p.err, MUON_ERR_TIMEOUT);
         *abort_flag = 1;
       }
-      // The first CTA's full barriers count both CTAs' bytes: waiting on them here
-      // means no copy of either CTA is still landing when the pair exits.
-      if (rank == 0)
+      // Never leave with bulk copies still landing in shared memory (for a pair, the
+      // first CTA's full barriers count both CTAs' bytes).
+      if (!PAIR || rank == 0)
         for (long long r = (q > S ? q - S : 0); r < q; ++r)
           mbar_wait(&full[r % S], static_cast<uint32_t>((r / S) & 1), nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (first CTA)
-    if (lane == 0 && rank == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(256, 256, B_MN);
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && (!PAIR || rank == 0)) {
+      const uint32_t idesc0 = idesc_bf16_f32(C::kMmaM, C::kMmaN, B_MN);
       long long q = 0;
       int it = 0;
       bool ok = true;
-      for (int t = cluster_id; t < total && ok; t += nclusters, ++it) {
+      for (int t = unit; t < total && ok; t += nunits, ++it) {
         const TileJob j = decode(p, t, SYM);
         const int kb_n = p.cls[j.c].k_blocks;
+        const int a_row0 = j.ti * C::kTileM;  // the first CTA's rows decide for both
+        const int b_row0 = j.tj * C::kTileN;
         const int ab = it & 1;
         const uint32_t apar = static_cast<uint32_t>((it >> 1) & 1);
         if (!mbar_wait(&tempty[ab], apar ^ 1u, abort_flag)) {
@@ -510,7 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * 256);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * C::kNCol);
         for (int kb = 0; kb < kb_n; ++kb) {
           const int s = static_cast<int>(q % S);
           const uint32_t par = static_cast<uint32_t>((q / S) & 1);
@@ -519,50 +288,67 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
             break;
           }
           tc_fence_after();
+          // one instruction serves both CTAs of a pair: the layout choice is made per
+          // cluster tile (block size kTileM), identical for both halves
+          const bool a_t = below_diag(A_SYM, a_row0, kb, C::kTileM);
+          const bool b_t = B_MN || below_diag(B_SYM, b_row0, kb, C::kTileN);
+          const uint32_t idesc = idesc0 | (a_t ? (1u << 15) : 0u) | (b_t ? (1u << 16) : 0u);
           const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
           const uint32_t sb = sa + C::kABytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 64 * BK * 2, 1024)
-                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
-            umma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t ad = op_desc(sa, kk, a_t);
+            const uint64_t bd = op_desc(sb, kk, b_t);
+            if (PAIR) umma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            else umma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
-          // the stage is free in both CTAs once these MMAs have read it
-          umma_commit_pair(smem_u32(&empty[s]));
-          umma_commit_pair(peer_addr(&empty[s], 1));
+          if (PAIR) {
+            umma_commit_pair(smem_u32(&empty[s]));
+            umma_commit_pair(peer_addr(&empty[s], 1));
+          } else {
+            umma_commit(&empty[s]);
+          }
           ++q;
         }
         if (!ok) break;
-        umma_commit_pair(smem_u32(&tfull[ab]));
-        umma_commit_pair(peer_addr(&tfull[ab], 1));
+        if (PAIR) {
+          umma_commit_pair(smem_u32(&tfull[ab]));
+          umma_commit_pair(peer_addr(&tfull[ab], 1));
+        } else {
+          umma_commit(&tfull[ab]);
+        }
       }
       if (!ok) {
         set_error(p.err, MUON_ERR_TIMEOUT);
         *abort_flag = 1;
       }
-      umma_commit_pair(smem_u32(done));
+      if (PAIR) umma_commit_pair(smem_u32(done));
+      else umma_commit(done);
       mbar_wait(done, 0, nullptr);
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-5, both CTAs)
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // row within this CTA's 128 rows
-    const bool leader = warp == 2 && lane == 0;
-    const int rk = static_cast<int>(rank);
+    // ------------------------------------------------------------ epilogue (warps 2-9)
+    const int ew = warp - 2;
+    const int quad = warp & 3;           // the TMEM lane quarter this warp may access
+    const int grp = ew >> 2;             // which half of each 128-column round
+    const int r = quad * 32 + lane;      // tile row of this thread within the CTA
+    const bool leader = ew == 0 && lane == 0;
     bool c_pending = false;
-    if (HAS_C && leader && cluster_id < total) {
-      const TileJob j = decode(p, cluster_id, SYM);
-      mbar_expect_tx(cfull, C::kCDBytes);
+    if (HAS_C && leader && unit < total) {
+      const TileJob j = decode(p, unit, SYM);
+      mbar_expect_tx(cfull, C::kStagingBytes);
 #pragma unroll
-      for (int h = 0; h < 4; ++h)
-        tma_load_3d(cd + h * (128 * 128), &P.tc[j.c], cfull, j.tj * 256 + h * 64, j.ti * 256 + rk * 128,
-                    j.mat);
+      for (int h = 0; h < C::kNCol / 64; ++h)
+        tma_load_3d(stg + h * (BM * 128), &P.tc[j.c], cfull, j.tj * C::kTileN + h * 64,
+                    j.ti * C::kTileM + rank * 128, j.mat);
       c_pending = true;
     }
+    // All epilogue warps walk the same tiles and execute every named barrier, also
+    // after a failed wait (they then skip the work): no warp is ever left waiting at
+    // a barrier.
     int it = 0;
     bool ok = true;
-    for (int t = cluster_id; t < total; t += nclusters, ++it) {
+    for (int t = unit; t < total; t += nunits, ++it) {
       const TileJob j = decode(p, t, SYM);
       const NsClassArgs& k = p.cls[j.c];
       const int ab = it & 1;
@@ -578,15 +364,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
       }
       const int m = k.m;
       const int ncols = PHASE == PH_APPLY ? k.n : m;
-      const int row0 = j.ti * 256 + rk * 128;
-      const int si = 2 * j.ti + rk;
-      bool direct[2], mirror[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int sj = 2 * j.tj + h;
-        direct[h] = (!SYM || sj >= si) && row0 < m && sj * 128 < ncols;
-        mirror[h] = SYM && sj > si && row0 < m && sj * 128 < m;
-      }
+      const int row0 = j.ti * C::kTileM + rank * 128;   // this CTA's first output row
+      const int col0 = j.tj * C::kTileN;                 // this CTA's first output column
       float scale = 1.f;
       if (ok) {
         if (leader) c_pending = false;
@@ -597,23 +376,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
         }
       }
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < C::kRounds; ++h) {
         if (ok) {
 #pragma unroll 1
-          for (int ch = 4 * h; ch < 4 * h + 4; ++ch) {
+          for (int ci = 0; ci < 2; ++ci) {
+            const int ch = 4 * h + 2 * grp + ci;   // 32-column chunk of the accumulator
             uint32_t v[32];
             tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                          static_cast<uint32_t>(ab * 256 + ch * 32),
+                          static_cast<uint32_t>(ab * C::kNCol + ch * 32),
                       v);
             tmem_wait_ld();
-            uint32_t packed[16];
-            const int dcol = (row0 + r) - (j.tj * 256 + ch * 32);
+            // the element of this row on the global diagonal, as a column of this chunk
+            const int dcol = (row0 + r) - (col0 + ch * 32);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
-              const uint32_t off = sw128_off(r, ch * 32 + q4 * 8);
+              const uint32_t off = HAS_C ? sw128_off(r, ch * 32 + q4 * 8)
+                                         : sw128_off(r, (ch - 4 * h) * 32 + q4 * 8);
               uint4 cw = make_uint4(0, 0, 0, 0);
-              if (HAS_C) cw = *reinterpret_cast<const uint4*>(cd + off);
+              if (HAS_C) cw = *reinterpret_cast<const uint4*>(stg + off);
               const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
+              uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
                 const int i0 = q4 * 8 + 2 * e;
@@ -627,55 +409,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
                   a0 *= scale;
                   a1 *= scale;
                 }
-                packed[q4 * 4 + e] = pack_bf16x2(a0, a1);
+                pk[e] = pack_bf16x2(a0, a1);
               }
-              *reinterpret_cast<uint4*>(cd + off) = make_uint4(
-                  packed[q4 * 4], packed[q4 * 4 + 1], packed[q4 * 4 + 2], packed[q4 * 4 + 3]);
-            }
-            if (mirror[h]) {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                *reinterpret_cast<uint16_t*>(tt + sw128_off((ch - 4 * h) * 32 + e, r)) =
-                    static_cast<uint16_t>(packed[e >> 1] >> ((e & 1) * 16));
+              *reinterpret_cast<uint4*>(stg + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           }
-          if (h == 1) {
-            // this CTA's accumulator rows have been read: free them for the MMA
+          if (h == C::kRounds - 1) {
+            // this warp has read its share of the accumulator: free it for the MMA
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-              if (rk == 0) mbar_arrive(&tempty[ab]);
+              if (!PAIR || rank == 0) mbar_arrive(&tempty[ab]);
               else mbar_arrive_cluster(peer_addr(&tempty[ab], 0));
             }
           }
           fence_proxy_async_smem();
         }
-        if (SYM || h == 1) {
+        if (!HAS_C || h == C::kRounds - 1) {
           named_barrier(1, kEpiWarps * 32);
+          if (leader && ok && row0 < m) {
+            // rounds of 128 columns (symmetric phases only compute tiles on or above
+            // the tile diagonal, and store all of them)
+            const int h0 = HAS_C ? 0 : h, h1 = HAS_C ? C::kRounds : h + 1;
+            for (int hh = h0; hh < h1; ++hh) {
+              const int cb = col0 + hh * 128;
+#pragma unroll
+              for (int b = 0; b < 2; ++b) {
+                const int x = cb + b * 64;
+                const uint8_t* src = stg + ((HAS_C ? hh * 2 : 0) + b) * (BM * 128);
+                if (x < ncols) tma_store_3d(&P.td[j.c], src, x, row0, j.mat);
+              }
+            }
+          }
           if (leader && ok) {
-            if (h == 1) {
-#pragma unroll
-              for (int b = 0; b < 4; ++b)
-                if (direct[b >> 1] && j.tj * 256 + b * 64 < ncols)
-                  tma_store_3d(&P.td[j.c], cd + b * (128 * 128), j.tj * 256 + b * 64, row0, j.mat);
-            }
-            if (mirror[h]) {
-              const int sj = 2 * j.tj + h;
-#pragma unroll
-              for (int b = 0; b < 2; ++b)
-                if (si * 128 + b * 64 < m)
-                  tma_store_3d(&P.td[j.c], tt + b * (128 * 128), si * 128 + b * 64, sj * 128, j.mat);
-            }
             tma_store_commit();
-            tma_store_wait_read();  // staging buffers are free again
-            const int tn = t + nclusters;
-            if (h == 1 && HAS_C && tn < total) {
+            tma_store_wait_read();  // the staging buffer is free again
+            const int tn = t + nunits;
+            if (HAS_C && tn < total) {
               const TileJob jn = decode(p, tn, SYM);
-              mbar_expect_tx(cfull, C::kCDBytes);
+              mbar_expect_tx(cfull, C::kStagingBytes);
 #pragma unroll
-              for (int b = 0; b < 4; ++b)
-                tma_load_3d(cd + b * (128 * 128), &P.tc[jn.c], cfull, jn.tj * 256 + b * 64,
-                            jn.ti * 256 + rk * 128, jn.mat);
+              for (int b = 0; b < C::kNCol / 64; ++b)
+                tma_load_3d(stg + b * (BM * 128), &P.tc[jn.c], cfull, jn.tj * C::kTileN + b * 64,
+                            jn.ti * C::kTileM + rank * 128, jn.mat);
               c_pending = true;
             }
           }
@@ -685,44 +461,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreadsTc, 1)
     }
     if (leader) {
       tma_store_wait_all();
-      if (c_pending) mbar_wait(cfull, it & 1, nullptr);
+      if (c_pending) mbar_wait(cfull, it & 1, nullptr);  // a C tile still landing
     }
   }
 
   __syncthreads();
-  cluster_sync_all();  // no cross-CTA signal or TMEM access is outstanding past this point
+  if (PAIR) cluster_sync_all();  // no cross-CTA signal or TMEM access outstanding
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    if (PAIR) tmem_dealloc_pair(tmem_base, C::kTmemCols);
+    else tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
-template <int PHASE>
-cudaError_t launch_pair(const TcParams& P, int grid, cudaStream_t s) {
+template <int BN, int PHASE, bool PAIR>
+cudaError_t launch_tc(const TcParams& P, int grid, cudaStream_t s) {
+  using C = TcCfg<BN, PHASE, PAIR>;
   static bool attr_set = false;
+  auto kern = ns_tc_kernel<BN, PHASE, PAIR>;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_tc_pair_kernel<PHASE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         PairCfg<PHASE>::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  ns_tc_pair_kernel<PHASE><<<grid, kThreadsTc, PairCfg<PHASE>::kSmemBytes, s>>>(P);
-  return cudaGetLastError();
-}
-
-template <int BN, int PHASE>
-cudaError_t launch_one(const TcParams& P, int grid, cudaStream_t s) {
-  using C = TcCfg<BN, PHASE>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_tc_kernel<BN, PHASE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
+  if (!PAIR) {
+    kern<<<grid, kThreadsTc, C::kSmemBytes, s>>>(P);
+    return cudaGetLastError();
   }
-  ns_tc_kernel<BN, PHASE><<<grid, kThreadsTc, C::kSmemBytes, s>>>(P);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
 }  // namespace
@@ -736,9 +515,9 @@ cudaError_t launch_ns_phase_tc_pair(const TcParams& P, int num_sms, cudaStream_t
   if (total <= 0) return cudaSuccess;
   const int pairs = total < num_sms / 2 ? total : num_sms / 2;
   switch (P.args.phase) {
-    case PH_GRAM: return launch_pair<PH_GRAM>(P, 2 * pairs, s);
-    case PH_POLY: return launch_pair<PH_POLY>(P, 2 * pairs, s);
-    default: return launch_pair<PH_APPLY>(P, 2 * pairs, s);
+    case PH_GRAM: return launch_tc<256, PH_GRAM, true>(P, 2 * pairs, s);
+    case PH_POLY: return launch_tc<256, PH_POLY, true>(P, 2 * pairs, s);
+    default: return launch_tc<256, PH_APPLY, true>(P, 2 * pairs, s);
   }
 }
 
@@ -747,9 +526,9 @@ cudaError_t launch_ns_phase_tc(const TcParams& P, int num_sms, cudaStream_t s) {
   if (total <= 0) return cudaSuccess;
   const int grid = total < num_sms ? total : num_sms;
   switch (P.args.phase) {
-    case PH_GRAM: return launch_one<128, PH_GRAM>(P, grid, s);
-    case PH_POLY: return launch_one<128, PH_POLY>(P, grid, s);
-    default: return launch_one<256, PH_APPLY>(P, grid, s);
+    case PH_GRAM: return launch_tc<128, PH_GRAM, false>(P, grid, s);
+    case PH_POLY: return launch_tc<128, PH_POLY, false>(P, grid, s);
+    default: return launch_tc<256, PH_APPLY, false>(P, grid, s);
   }
 }
 

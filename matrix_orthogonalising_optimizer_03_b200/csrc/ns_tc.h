@@ -11,12 +11,15 @@ namespace muon {
 // epilogue's C tile and of the output, plus the phase arguments. Passed as a __grid_constant__ parameter so
 // the TMA unit reads the maps from parameter space.
 struct TcParams {
-  CUtensorMap ta[kMaxClassesPerLaunch];  // A operand (64 x 128 boxes)
-  CUtensorMap tb[kMaxClassesPerLaunch];  // B operand
-  CUtensorMap tc[kMaxClassesPerLaunch];  // C tile of the epilogue (POLY: S, APPLY: X)
-  CUtensorMap td[kMaxClassesPerLaunch];  // output (GRAM: S, POLY: P, APPLY: X')
+  CUtensorMap ta[kMaxClassesPerLaunch];    // A operand, K-major 64 x 128 boxes
+  CUtensorMap ta_t[kMaxClassesPerLaunch];  // A operand mirror blocks, 64 x 64 boxes
+  CUtensorMap tb[kMaxClassesPerLaunch];    // B operand (APPLY: X, 64 x 64 boxes)
+  CUtensorMap tb_t[kMaxClassesPerLaunch];  // B operand mirror blocks (POLY), 64 x 64 boxes
+  CUtensorMap tc[kMaxClassesPerLaunch];    // C tile of the epilogue (POLY: S)
+  CUtensorMap td[kMaxClassesPerLaunch];    // output (GRAM: S, POLY: P', APPLY: X'), 64 x 128
   NsPhaseArgs args;
 };
+static_assert(sizeof(TcParams) <= 4096, "kernel parameters must fit the portable 4 KB");
 
 // Tile sizes of the tensor-core phases (rows x cols of an output tile, k-block).
 int tc_block_m();

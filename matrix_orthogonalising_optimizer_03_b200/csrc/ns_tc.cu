@@ -66,7 +66,7 @@ struct TcCfg {
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = kBRows * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStagingBytes = kHasC ? BM * kNCol * 2 : BM * 128 * 2;
+  static constexpr int kStagingBytes = kHasC ? BM * kNCol * 2 : 2 * BM * 64 * 2;  // C tile, or 2 x 16 KB
   static constexpr int kBudget = 224 * 1024;
   static constexpr int kFit = (kBudget - kStagingBytes) / kStageBytes;
   static constexpr int kStages = kFit > 8 ? 8 : kFit;
@@ -78,8 +78,7 @@ struct TcCfg {
   static constexpr int kMmaN = PAIR ? 256 : BN;
   static constexpr int kTileM = PAIR ? 256 : 128;          // output tile (cluster) rows
   static constexpr int kTileN = PAIR ? 256 : BN;           // output tile columns
-  static constexpr int kChunks = kNCol / 32;               // 32-column TMEM chunks per CTA
-  static constexpr int kRounds = kNCol / 128;              // 128-column store rounds
+  static constexpr int kRounds = kHasC ? 1 : kNCol / 64;   // output rounds (64 columns each)
   static_assert(kStages >= 3, "pipeline too shallow");
 };
 
@@ -143,12 +142,6 @@ __device__ __forceinline__ void load_k_block(uint8_t* dst, const CUtensorMap* mk
       else tma_load_3d(dst + h * (64 * BK * 2), mt, bar, row0 + h * 64, kb * BK, mat);
     }
   }
-}
-
-// Descriptor of the kk-th K = 16 slice of a staged operand block.
-__device__ __forceinline__ uint64_t op_desc(uint32_t base, int kk, bool mn_major) {
-  return mn_major ? smem_desc_sw128(base + kk * 2048, 64 * BK * 2, 1024)
-                  : smem_desc_sw128(base + kk * 32, 16, 1024);
 }
 
 template <int BN, int PHASE, bool PAIR>
@@ -264,6 +257,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && (!PAIR || rank == 0)) {
       const uint32_t idesc0 = idesc_bf16_f32(C::kMmaM, C::kMmaN, B_MN);
+      // descriptors differ per k-slice only in the start-address field: build the
+      // constant part once (K-major: LBO 16 B; MN-major: LBO 8 KB between 64-element
+      // chunks; both SBO 1024 B) and add the address per slice
+      const uint64_t kmaj_hi = smem_desc_sw128(0, 16, 1024);
+      const uint64_t mnmaj_hi = smem_desc_sw128(0, 64 * BK * 2, 1024);
       long long q = 0;
       int it = 0;
       bool ok = true;
@@ -295,10 +293,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           const uint32_t idesc = idesc0 | (a_t ? (1u << 15) : 0u) | (b_t ? (1u << 16) : 0u);
           const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
           const uint32_t sb = sa + C::kABytes;
+          // K-major slices advance 32 B (2 in the >>4 address field), MN-major 2 KB (128)
+          const uint64_t ad0 = (a_t ? mnmaj_hi : kmaj_hi) | static_cast<uint64_t>((sa >> 4) & 0x3FFFu);
+          const uint64_t bd0 = (b_t ? mnmaj_hi : kmaj_hi) | static_cast<uint64_t>((sb >> 4) & 0x3FFFu);
+          const uint64_t astep = a_t ? 128u : 2u, bstep = b_t ? 128u : 2u;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = op_desc(sa, kk, a_t);
-            const uint64_t bd = op_desc(sb, kk, b_t);
+            const uint64_t ad = ad0 + astep * kk;
+            const uint64_t bd = bd0 + bstep * kk;
             if (PAIR) umma_f16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
             else umma_f16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
           }
@@ -375,12 +377,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           scale = static_cast<float>(PHASE == PH_GRAM ? inv * inv : inv);
         }
       }
+      // Output rounds. POLY writes D over its C tile and stores it whole after the
+      // last round; GRAM / APPLY stage 64 columns per round in two alternating 16 KB
+      // buffers, so a round's store overlaps the next round's math.
 #pragma unroll 1
-      for (int h = 0; h < C::kRounds; ++h) {
+      for (int rr = 0; rr < C::kRounds; ++rr) {
         if (ok) {
 #pragma unroll 1
-          for (int ci = 0; ci < 2; ++ci) {
-            const int ch = 4 * h + 2 * grp + ci;   // 32-column chunk of the accumulator
+          for (int ci = 0; ci < (HAS_C ? C::kNCol / 64 : 1); ++ci) {
+            const int ch = HAS_C ? 2 * ci + grp : 2 * rr + grp;   // 32-column accumulator chunk
             uint32_t v[32];
             tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                           static_cast<uint32_t>(ab * C::kNCol + ch * 32),
@@ -388,12 +393,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
             tmem_wait_ld();
             // the element of this row on the global diagonal, as a column of this chunk
             const int dcol = (row0 + r) - (col0 + ch * 32);
+            uint8_t* buf = HAS_C ? stg : stg + (rr & 1) * (BM * 128);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               const uint32_t off = HAS_C ? sw128_off(r, ch * 32 + q4 * 8)
-                                         : sw128_off(r, (ch - 4 * h) * 32 + q4 * 8);
+                                         : sw128_off(r, grp * 32 + q4 * 8);
               uint4 cw = make_uint4(0, 0, 0, 0);
-              if (HAS_C) cw = *reinterpret_cast<const uint4*>(stg + off);
+              if (HAS_C) cw = *reinterpret_cast<const uint4*>(buf + off);
               const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
               uint32_t pk[4];
 #pragma unroll
@@ -411,10 +417,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
                 }
                 pk[e] = pack_bf16x2(a0, a1);
               }
-              *reinterpret_cast<uint4*>(stg + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              *reinterpret_cast<uint4*>(buf + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
           }
-          if (h == C::kRounds - 1) {
+          if (rr == C::kRounds - 1) {
             // this warp has read its share of the accumulator: free it for the MMA
             tc_fence_before();
             __syncwarp();
@@ -425,27 +431,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           }
           fence_proxy_async_smem();
         }
-        if (!HAS_C || h == C::kRounds - 1) {
-          named_barrier(1, kEpiWarps * 32);
-          if (leader && ok && row0 < m) {
-            // rounds of 128 columns (symmetric phases only compute tiles on or above
-            // the tile diagonal, and store all of them)
-            const int h0 = HAS_C ? 0 : h, h1 = HAS_C ? C::kRounds : h + 1;
-            for (int hh = h0; hh < h1; ++hh) {
-              const int cb = col0 + hh * 128;
+        named_barrier(1, kEpiWarps * 32);
+        if (leader && ok) {
+          if (HAS_C) {
+            if (row0 < m) {
 #pragma unroll
-              for (int b = 0; b < 2; ++b) {
-                const int x = cb + b * 64;
-                const uint8_t* src = stg + ((HAS_C ? hh * 2 : 0) + b) * (BM * 128);
-                if (x < ncols) tma_store_3d(&P.td[j.c], src, x, row0, j.mat);
-              }
+              for (int b = 0; b < C::kNCol / 64; ++b)
+                if (col0 + b * 64 < ncols)
+                  tma_store_3d(&P.td[j.c], stg + b * (BM * 128), col0 + b * 64, row0, j.mat);
             }
-          }
-          if (leader && ok) {
             tma_store_commit();
-            tma_store_wait_read();  // the staging buffer is free again
+            tma_store_wait_read();  // the C / D buffer is free again
             const int tn = t + nunits;
-            if (HAS_C && tn < total) {
+            if (tn < total) {
               const TileJob jn = decode(p, tn, SYM);
               mbar_expect_tx(cfull, C::kStagingBytes);
 #pragma unroll
@@ -454,9 +452,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
                             jn.ti * C::kTileM + rank * 128, jn.mat);
               c_pending = true;
             }
+          } else {
+            const int x = col0 + rr * 64;
+            if (row0 < m && x < ncols)
+              tma_store_3d(&P.td[j.c], stg + (rr & 1) * (BM * 128), x, row0, j.mat);
+            tma_store_commit();
+            tma_store_wait_read_1();  // the previous round's buffer is free again
           }
-          named_barrier(1, kEpiWarps * 32);
         }
+        named_barrier(1, kEpiWarps * 32);
       }
     }
     if (leader) {

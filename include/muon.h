@@ -79,7 +79,20 @@ typedef enum { MUON_F32 = 0, MUON_BF16 = 1 } muon_dtype_t;
 
 typedef enum {
   MUON_MODE_MUON = 0,    /* plain Muon (with decoupled weight decay when wd > 0) */
-  MUON_MODE_MUONGS = 1   /* MuonGS: radial (Gram-Schmidt) projection before the update */
+  MUON_MODE_MUONGS = 1,  /* MuonGS: radial (Gram-Schmidt) projection before the update */
+  MUON_MODE_MUONH = 2,   /* MuonH: fixed radius, W_{t+1} = ||W_t|| W' / ||W'|| with W' the
+                            plain Muon update ("MuonGS: Pretraining LLMs with Relaxed
+                            Weight-Norm Control", section 무엇과 다른가, names fixed-norm
+                            control; the retraction form is this library's reading) */
+  MUON_MODE_TWOSIDED = 3 /* for 2-D parameters that are not orthogonalised ("행과 열을 함께
+                            정규화하는 ... MeqMuon 공개", section 핵심 내용): no Newton-Schulz;
+                            the Frobenius-normalised Nesterov direction X is normalised along
+                            rows and columns at once, N_ij = X_ij rho / ((sqrt(r_i)+eps)
+                            (sqrt(c_j)+eps)), r / c the row / column mean squares of X and rho
+                            its RMS (this library's reading; no formula on the page). Use
+                            scale MUON_SCALE_NONE for an update of RMS about 1. ns_steps and
+                            MUON_EQUILIBRATE are ignored; stats report w_norm only (the
+                            other fields are NaN). */
 } muon_mode_t;
 
 typedef enum {
@@ -232,6 +245,27 @@ MUON_API int muon_plan_profile_read(muon_plan_t plan, muon_profile_entry_t* out,
 MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matrix_t* mat,
                                                   const muon_hparams_t* hp, uint32_t* status_dev,
                                                   void* stream);
+
+/* ---- QK-Clip (MuonClip) ----
+ * "LLM Pretraining Loss Spike 진단과 처방", section "Moonlight와 MuonClip이 추가한 것"
+ * (QK-Clip listing): for attention head h whose largest pre-softmax logit S_max[h]
+ * exceeds tau, gamma_h = tau / S_max[h] (else 1); the head's non-rotary query and key
+ * projection rows are multiplied by gamma_h^0.5, its rotary query rows by gamma_h,
+ * and the rotary key shared by all heads is not touched.
+ * A slice names rows [row0, row0 + rows) of a row-major fp32 device matrix W (all
+ * `cols` columns, leading dimension ld) that belong to head `head` and are scaled by
+ * gamma_head^power (0.5 or 1.0 in the listing). s_max_dev: device array of n_heads
+ * floats (the caller's forward pass measures them). Slices of one call may not
+ * overlap (MUON_ERR_ALIAS). Asynchronous on `stream`; no workspace. */
+typedef struct {
+  void* W;
+  int64_t row0, rows, cols, ld;
+  int32_t head;
+  float power;
+} muon_qk_slice_t;
+
+MUON_API muon_status_t muon_qk_clip(const muon_qk_slice_t* slices, int n, const float* s_max_dev,
+                                    int n_heads, float tau, void* stream);
 
 /* Self-test of the device-side timeout path: launches one thread that waits, with
  * the same bounded wait the pipelined kernels use, on an mbarrier nothing arrives

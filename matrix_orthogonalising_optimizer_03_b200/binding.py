@@ -22,11 +22,12 @@ STATUS_NAMES = {
     8: "MUON_ERR_UNSUPPORTED",
 }
 MUON_F32, MUON_BF16 = 0, 1
-MUON_MODE_MUON, MUON_MODE_MUONGS = 0, 1
+MUON_MODE_MUON, MUON_MODE_MUONGS, MUON_MODE_MUONH, MUON_MODE_TWOSIDED = 0, 1, 2, 3
 MUON_SCALE_MOONLIGHT, MUON_SCALE_KELLER, MUON_SCALE_NONE = 0, 1, 2
 MUON_NESTEROV, MUON_EQUILIBRATE, MUON_NS_FP32, MUON_WANT_STATS = 1, 2, 4, 8
 
-MODES = {"muon": MUON_MODE_MUON, "muongs": MUON_MODE_MUONGS}
+MODES = {"muon": MUON_MODE_MUON, "muongs": MUON_MODE_MUONGS, "muonh": MUON_MODE_MUONH,
+         "twosided": MUON_MODE_TWOSIDED}
 SCALES = {"moonlight": MUON_SCALE_MOONLIGHT, "keller": MUON_SCALE_KELLER, "none": MUON_SCALE_NONE}
 
 
@@ -53,6 +54,11 @@ class MuonHParams(ctypes.Structure):
 class MuonStats(ctypes.Structure):
     _fields_ = [("w_norm", c_float), ("w_dot_o", c_float), ("o_norm", c_float),
                 ("update_rms", c_float), ("equil_axis", c_int32), ("reserved", c_int32)]
+
+
+class MuonQkSlice(ctypes.Structure):
+    _fields_ = [("W", c_void_p), ("row0", c_int64), ("rows", c_int64), ("cols", c_int64),
+                ("ld", c_int64), ("head", c_int32), ("power", c_float)]
 
 
 class MuonNSMatrix(ctypes.Structure):
@@ -93,6 +99,7 @@ def load(path: str = LIB_PATH):
         "muon_newton_schulz_noalloc": (c_int, [P(MuonNSMatrix), P(MuonHParams), c_void_p, c_void_p]),
         "muon_plan_profile_enable": (c_int, [c_void_p, c_int]),
         "muon_wait_probe": (c_int, [c_void_p, c_int64, c_void_p]),
+        "muon_qk_clip": (c_int, [P(MuonQkSlice), c_int, c_void_p, c_int, c_float, c_void_p]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -298,3 +305,19 @@ def newton_schulz_noalloc(x, o, hp: MuonHParams, status=None, stream=None):
     _check(lib.muon_newton_schulz_noalloc(ctypes.byref(m), ctypes.byref(hp),
                                           status.data_ptr() if status is not None else None,
                                           _stream_ptr(stream)), "muon_newton_schulz_noalloc")
+
+
+def qk_clip(slices, s_max, tau: float = 100.0, stream=None):
+    """QK-Clip. slices: list of (W tensor fp32 2-D CUDA, row0, rows, head, power);
+    s_max: CUDA float32 tensor with one entry per head."""
+    lib = load()
+    arr = (MuonQkSlice * len(slices))()
+    for i, (w, r0, nr, h, pw) in enumerate(slices):
+        _check_2d(w, "W")
+        if w.dtype != _torch().float32:
+            raise MuonError(3, "QK-Clip weights must be float32")
+        arr[i] = MuonQkSlice(w.data_ptr(), r0, nr, w.size(1), max(w.stride(0), w.size(1)), h, pw)
+    if s_max.dtype != _torch().float32 or not s_max.is_cuda:
+        raise MuonError(1, "s_max must be a CUDA float32 tensor")
+    _check(lib.muon_qk_clip(arr, len(slices), s_max.data_ptr(), s_max.numel(), tau,
+                            _stream_ptr(stream)), "muon_qk_clip")

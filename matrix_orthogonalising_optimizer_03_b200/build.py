@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmuon.so")
 
-SOURCES = ["muon_api.cpp", "elementwise.cu", "ns_simt.cu", "ns_tc.cu", "noalloc.cu", "diagnostics.cu"]
+SOURCES = ["muon_api.cpp", "elementwise.cu", "ns_simt.cu", "ns_tc.cu", "noalloc.cu", "diagnostics.cu", "qkclip.cu"]
 HEADERS = ["muon_internal.h", "ptx.cuh", "ns_tc.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

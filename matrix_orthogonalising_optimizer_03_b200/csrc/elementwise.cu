@@ -358,6 +358,36 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
 
   double wdo = sc.wo, doo = sc.o2;  // <W, D O>, ||D O||^2
   int axis = 0;
+  if (a.mode == MUON_MODE_TWOSIDED) {
+    // N_ij = X_ij rho / ((sqrt(r_i)+eps)(sqrt(c_j)+eps)): the row factor (with rho)
+    // and the column factor go to the two halves of eq_o2
+    const double rho = sqrt(sc.o2 / (rows * cols));
+    for (int i = threadIdx.x; i < d.rows; i += kThreads)
+      a.eq_o2[s.eq_off + i] =
+          static_cast<float>(rho / (sqrt((double)a.eq_o2[s.eq_off + i] / cols) + (double)a.eps));
+    for (int j = threadIdx.x; j < d.cols; j += kThreads)
+      a.eq_o2[s.eq_off + d.rows + j] = static_cast<float>(
+          1.0 / (sqrt((double)a.eq_o2[s.eq_off + d.rows + j] / rows) + (double)a.eps));
+    if (threadIdx.x != 0) return;
+    MatCoef cf;
+    cf.cw = static_cast<float>(1.0 - (double)a.lr * (double)a.wd);
+    cf.co = static_cast<float>(-(double)a.lr * scale);
+    cf.axis = 3;
+    cf.pad = 0;
+    a.coef[k] = cf;
+    if (a.stats != nullptr) {
+      const float nan = __int_as_float(0x7fc00000);
+      muon_stats_t st;
+      st.w_norm = static_cast<float>(sqrt(sc.w2));
+      st.w_dot_o = nan;
+      st.o_norm = nan;
+      st.update_rms = nan;
+      st.equil_axis = 3;
+      st.reserved = 0;
+      a.stats[d.orig] = st;
+    }
+    return;
+  }
   if (a.equilibrate) {
     // imbalance = std / mean of the row RMS and of the column RMS vectors
     double sr = 0, sr2 = 0, scs = 0, sc2 = 0;
@@ -396,11 +426,20 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
   if (threadIdx.x != 0) return;
   wdo *= scale;                 // <W, O> with O = s*D*O_raw
   const double oo = scale * scale * doo;
+  const double lr = a.lr, cw0 = 1.0 - lr * (double)a.wd;
   double g = 0.0;
   if (a.mode == MUON_MODE_MUONGS && sc.w2 > 0.0) g = wdo / sc.w2;
+  double cw = cw0 + lr * g, co = -lr * scale;
+  if (a.mode == MUON_MODE_MUONH) {
+    // W' = cw0 W - lr O; rescale to the current radius ||W_t||
+    const double n2 = cw0 * cw0 * sc.w2 - 2.0 * cw0 * lr * wdo + lr * lr * oo;
+    const double f = n2 > 0.0 ? sqrt(sc.w2 / n2) : 1.0;
+    cw *= f;
+    co *= f;
+  }
   MatCoef cf;
-  cf.cw = static_cast<float>(1.0 - (double)a.lr * (double)a.wd + (double)a.lr * g);
-  cf.co = static_cast<float>(-(double)a.lr * scale);
+  cf.cw = static_cast<float>(cw);
+  cf.co = static_cast<float>(co);
   cf.axis = axis;
   cf.pad = 0;
   a.coef[k] = cf;
@@ -453,11 +492,11 @@ __global__ void __launch_bounds__(kThreads, 6) post_apply_kernel(const ElemArgs 
       float w[8];
       float* wp = d.W + (int64_t)r * d.ld_w + c;
       load8_f32(wp, vec, valid, w);
-      const float rowf = cf.axis == 1 ? a.eq_o2[s.eq_off + r] : 1.f;
+      const float rowf = (cf.axis & 1) ? a.eq_o2[s.eq_off + r] : 1.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         float f = xs * rowf;
-        if (cf.axis == 2 && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+        if ((cf.axis & 2) && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
         w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
       }
       store8_f32(wp, vec, valid, w);

@@ -46,6 +46,7 @@ struct muon_plan_s {
   bool ns_only = false;
   int n = 0;
   muon_hparams_t hp{};
+  int ns_steps = 0;  // Newton-Schulz iterations actually run (0 in the two-sided mode)
   bool x_fp32 = false;
   bool equilibrate = false;
   std::vector<ClassInfo> classes;
@@ -82,7 +83,9 @@ namespace {
 
 bool valid_enum_hp(const muon_hparams_t* hp) {
   if (hp->ns_steps < 0 || hp->ns_steps > 64) return false;
-  if (hp->mode != MUON_MODE_MUON && hp->mode != MUON_MODE_MUONGS) return false;
+  if (hp->mode != MUON_MODE_MUON && hp->mode != MUON_MODE_MUONGS && hp->mode != MUON_MODE_MUONH &&
+      hp->mode != MUON_MODE_TWOSIDED)
+    return false;
   if (hp->scale != MUON_SCALE_MOONLIGHT && hp->scale != MUON_SCALE_KELLER &&
       hp->scale != MUON_SCALE_NONE)
     return false;
@@ -232,7 +235,7 @@ void build_plan(muon_plan_s* p) {
   p->off_eq_o2 = off;  off = align_up(off + sizeof(float) * p->eq_total, kAlign);
   p->off_eq_wo = off;  off = align_up(off + sizeof(float) * p->eq_total, kAlign);
   off = align_up(off, kSlabAlign);
-  const bool two_x = p->hp.ns_steps > 0;
+  const bool two_x = p->ns_steps > 0;
   for (ClassInfo& ci : p->classes) {
     ci.off_x[0] = static_cast<int64_t>(off);
     off = align_up(off + ci.xbytes * ci.count, kSlabAlign);
@@ -242,7 +245,7 @@ void build_plan(muon_plan_s* p) {
     } else {
       ci.off_x[1] = ci.off_x[0];
     }
-    if (p->hp.ns_steps > 0) {
+    if (p->ns_steps > 0) {
       ci.off_s = static_cast<int64_t>(off);
       off = align_up(off + ci.sbytes * ci.count, kSlabAlign);
       ci.off_p = static_cast<int64_t>(off);
@@ -269,8 +272,11 @@ muon_plan_s* make_step_plan(const muon_matrix_t* mats, int n, const muon_hparams
   p->ns_only = false;
   p->n = n;
   p->hp = *hp;
-  p->x_fp32 = (hp->flags & MUON_NS_FP32) != 0;
-  p->equilibrate = (hp->flags & MUON_EQUILIBRATE) != 0;
+  const bool two_sided = hp->mode == MUON_MODE_TWOSIDED;
+  p->ns_steps = two_sided ? 0 : hp->ns_steps;
+  // the two-sided mode keeps U in fp32 and needs the row / column sums
+  p->x_fp32 = (hp->flags & MUON_NS_FP32) != 0 || two_sided;
+  p->equilibrate = (hp->flags & MUON_EQUILIBRATE) != 0 || two_sided;
   p->dev.resize(n);
   for (int i = 0; i < n; ++i) {
     const muon_matrix_t& m = mats[i];
@@ -299,6 +305,7 @@ muon_plan_s* make_ns_plan(const muon_ns_matrix_t* mats, int n, const muon_hparam
   p->ns_only = true;
   p->n = n;
   p->hp = *hp;
+  p->ns_steps = hp->ns_steps;
   p->x_fp32 = (hp->flags & MUON_NS_FP32) != 0;
   p->equilibrate = false;
   p->dev.resize(n);
@@ -354,7 +361,7 @@ muon_status_t current_device(int* dev, int* num_sms) {
 muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t stream) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int n = p->n;
-  const int steps = p->hp.ns_steps;
+  const int steps = p->ns_steps;
   std::vector<DevSlab> slabs(n);
   for (size_t c = 0; c < p->classes.size(); ++c) {
     const ClassInfo& ci = p->classes[c];
@@ -535,7 +542,7 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
   ea.ns_only = p->ns_only ? 1 : 0;
   ea.x_fp32 = p->x_fp32 ? 1 : 0;
   ea.equilibrate = p->equilibrate ? 1 : 0;
-  ea.xs_from_u2 = hp.ns_steps == 0 ? 1 : 0;
+  ea.xs_from_u2 = p->ns_steps == 0 ? 1 : 0;
 
   {
     ProfScope ps(p, stream);
@@ -545,7 +552,7 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
 
   // Newton-Schulz phases, at most kMaxClassesPerLaunch classes per launch
   const int nc = static_cast<int>(p->classes.size());
-  for (int it = 0; it < hp.ns_steps; ++it) {
+  for (int it = 0; it < p->ns_steps; ++it) {
     for (int phase = PH_GRAM; phase <= PH_APPLY; ++phase) {
       for (int c0 = 0; p->x_fp32 && c0 < nc; c0 += kMaxClassesPerLaunch) {
         const int cn = std::min(kMaxClassesPerLaunch, nc - c0);
@@ -640,7 +647,7 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
   }
 
   if (!p->ns_only) {
-    const bool need_reduce = hp.mode == MUON_MODE_MUONGS || p->equilibrate || stats != nullptr;
+    const bool need_reduce = hp.mode != MUON_MODE_MUON || p->equilibrate || stats != nullptr;
     if (need_reduce) {
       ProfScope ps(p, stream);
       if (launch_post_reduce(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
@@ -738,9 +745,13 @@ muon_status_t muon_plan_set_hparams(muon_plan_t plan, const muon_hparams_t* hp) 
   if (plan == nullptr || hp == nullptr || !valid_enum_hp(hp)) return MUON_ERR_INVALID_ARG;
   const uint32_t layout = MUON_NS_FP32 | MUON_EQUILIBRATE;
   if ((hp->flags & layout) != (plan->hp.flags & layout)) return MUON_ERR_INVALID_ARG;
-  if ((hp->ns_steps == 0) != (plan->hp.ns_steps == 0)) return MUON_ERR_INVALID_ARG;
-  const bool parity_changed = (hp->ns_steps % 2) != (plan->hp.ns_steps % 2);
+  if ((hp->mode == MUON_MODE_TWOSIDED) != (plan->hp.mode == MUON_MODE_TWOSIDED))
+    return MUON_ERR_INVALID_ARG;
+  const int steps = hp->mode == MUON_MODE_TWOSIDED ? 0 : hp->ns_steps;
+  if ((steps == 0) != (plan->ns_steps == 0)) return MUON_ERR_INVALID_ARG;
+  const bool parity_changed = (steps % 2) != (plan->ns_steps % 2);
   plan->hp = *hp;
+  plan->ns_steps = steps;
   if (parity_changed) plan->ws_cached = nullptr;  // the result slab moved: re-upload
   return MUON_OK;
 }

@@ -33,6 +33,11 @@ Readings where the pages are silent (each one also listed in the design notes):
   * equilibration: stateless row-or-column RMS balancing (see `equilibrate`).
     PARITY UNPINNED beyond the invariants its tests check: the pages give no formula.
   * GS projection is skipped when ||W||_F = 0.
+  * MuonH (fixed-radius control, named in [P2]): W_{t+1} = ||W_t|| W' / ||W'||,
+    W' the plain Muon update; the radius carries over, so it stays ||W_0||.
+  * two-sided normalisation ([P4], MeqMuon's treatment of the 2-D parameters that
+    are not orthogonalised; no formula on the pages): see `two_sided_normalise`.
+    PARITY UNPINNED beyond its rank-one closed form.
 """
 from __future__ import annotations
 
@@ -60,7 +65,7 @@ class HParams:
     ns_coeffs: Tuple[float, float, float] = QUINTIC
     ns_steps: int = 5
     eps: float = 1e-7
-    mode: str = "muon"           # "muon" | "muongs"
+    mode: str = "muon"           # "muon" | "muongs" | "muonh" | "twosided"
     scale: str = "moonlight"     # "moonlight" | "keller" | "none"
     scale_k: float = 0.2
     equilibrate: bool = False
@@ -167,6 +172,21 @@ def equilibrate(O: np.ndarray, eps: float = 1e-7) -> Tuple[np.ndarray, int]:
     return O * (rho / (c + eps))[None, :], AXIS_COLS
 
 
+def two_sided_normalise(X: np.ndarray, eps: float = 1e-7) -> np.ndarray:
+    """Two-sided (row and column at once) normalisation of a momentum matrix, [P4]
+    section 핵심 내용: MeqMuon normalises the momentum of the 2-D parameters it does not
+    orthogonalise along both rows and columns, without storing a second moment. The
+    pages give no formula. Reading: with r_i and c_j the mean squares of row i and
+    column j and rho the RMS of X, N_ij = X_ij rho / ((sqrt(r_i) + eps)(sqrt(c_j) + eps)),
+    the rank-one (row x column) estimate of the second moment a second-moment
+    optimizer would divide by. A rank-one X = u v^T maps to sign(u) sign(v)^T.
+    PARITY UNPINNED beyond that closed form."""
+    r = np.mean(X * X, axis=1)
+    c = np.mean(X * X, axis=0)
+    rho = np.sqrt(np.mean(X * X))
+    return X * rho / ((np.sqrt(r) + eps)[:, None] * (np.sqrt(c) + eps)[None, :])
+
+
 # ---------------------------------------------------------------- step a7
 def update_scale(rows: int, cols: int, rule: str = "moonlight", k: float = 0.2) -> float:
     """Per-matrix update scale.
@@ -202,6 +222,14 @@ def apply_update(W: np.ndarray, O_tilde: np.ndarray, lr: float, wd: float) -> np
     return (1.0 - lr * wd) * W - lr * O_tilde
 
 
+def retract_to_radius(W_new: np.ndarray, radius: float) -> np.ndarray:
+    """MuonH's fixed-radius control ([P2] 무엇과 다른가: MuonH keeps the weight norm at a
+    fixed radius R, so C_T = eta T / R). The pages print no retraction; reading: rescale
+    the updated matrix back to the radius, W <- R W / ||W||, with R = ||W_t||."""
+    n = float(np.linalg.norm(W_new))
+    return W_new if n == 0.0 else (radius / n) * W_new
+
+
 # ---------------------------------------------------------------- whole step
 def muon_step(W: np.ndarray, G: np.ndarray, M_prev: np.ndarray, hp: HParams) -> StepResult:
     """One Muon / MuonGS step of one matrix, steps a1-a9 in the order of [P5] section 3:
@@ -214,16 +242,22 @@ def muon_step(W: np.ndarray, G: np.ndarray, M_prev: np.ndarray, hp: HParams) -> 
         raise ValueError("Muon takes 2-D matrices only")
     rows, cols = W.shape
     M, U = momentum(M_prev, G, hp.momentum, hp.nesterov)
-    O = orthogonalise(U, hp)
     axis = AXIS_NONE
-    if hp.equilibrate:
-        O, axis = equilibrate(O, hp.eps)
+    if hp.mode == "twosided":
+        O = two_sided_normalise(frobenius_normalise(U, hp.eps), hp.eps)
+        axis = 3
+    else:
+        O = orthogonalise(U, hp)
+        if hp.equilibrate:
+            O, axis = equilibrate(O, hp.eps)
     O = update_scale(rows, cols, hp.scale, hp.scale_k) * O
     w_norm = float(np.linalg.norm(W))
     w_dot_o = float(np.sum(W * O))
     O_tilde = gs_project(W, O) if hp.mode == "muongs" else O
     o_norm = float(np.linalg.norm(O_tilde))
     W_next = apply_update(W, O_tilde, hp.lr, hp.weight_decay)
+    if hp.mode == "muonh":
+        W_next = retract_to_radius(W_next, w_norm)
     return StepResult(W_next, M, O, O_tilde, w_norm, w_dot_o, o_norm,
                       o_norm / np.sqrt(rows * cols), axis)
 
@@ -261,3 +295,22 @@ def muonw_radius(r0: float, p: float, lam: float) -> float:
     """[P2] 무엇과 다른가: R_lambda = max{r0, sqrt(p)/lambda}; MuonW keeps ||W_t|| <= R_lambda
     and C_T >= eta T / R_lambda."""
     return max(r0, np.sqrt(p) / lam)
+
+
+# ---------------------------------------------------------------- QK-Clip
+def qk_clip(weights: Sequence[np.ndarray], slices: Sequence[Tuple[int, int, int, int, float]],
+            s_max: Sequence[float], tau: float = 100.0) -> List[np.ndarray]:
+    """QK-Clip of [P1] (section "Moonlight와 MuonClip이 추가한 것", the QK-Clip listing):
+    for each head h, gamma_h = min(1, tau / S_max[h]); the head's non-rotary query and
+    key projections are multiplied by gamma^0.5, its rotary query projection by gamma,
+    and the rotary key (shared by all heads) is left alone.
+
+    `slices` lists (weight index, first row, row count, head, power): rows
+    [first, first+count) of weights[index] belong to head `head` and are scaled by
+    gamma_head ** power (0.5 for non-rotary q / k, 1.0 for rotary q). Returns new arrays.
+    """
+    out = [np.array(w, dtype=np.float64, copy=True) for w in weights]
+    for wi, r0, nr, h, power in slices:
+        gamma = min(1.0, tau / s_max[h])
+        out[wi][r0:r0 + nr, :] *= gamma ** power
+    return out

@@ -272,3 +272,56 @@ def test_rank_one_input_closed_form():
     want = _scalar_quintic(x, 5) * np.outer(u / np.linalg.norm(u), v / np.linalg.norm(v))
     got = orc.orthogonalise(U, orc.HParams())
     assert np.abs(got - want).max() < 1e-14
+
+
+def test_muonh_keeps_the_radius_and_ct_is_linear():
+    """Fixed-norm control (MuonGS page, 무엇과 다른가): ||W_t|| = R for all t and
+    C_T = eta T / R exactly."""
+    rng = np.random.default_rng(13)
+    rows, cols, eta, T = 24, 40, 0.02, 50
+    W0 = rng.standard_normal((rows, cols)) * 0.02
+    R = np.linalg.norm(W0)
+    hp = orc.HParams(lr=eta, mode="muonh", weight_decay=0.1)
+    res = orc.muon_run(W0, [rng.standard_normal((rows, cols)) * 1e-3 for _ in range(T)], hp)
+    assert all(abs(r.w_norm - R) <= 1e-12 * R for r in res)
+    assert abs(np.linalg.norm(res[-1].W) - R) <= 1e-12 * R
+    assert orc.accumulated_lr([eta] * T, [r.w_norm for r in res]) == pytest.approx(eta * T / R, rel=1e-12)
+    # one step by hand: the plain Muon update rescaled to ||W_0||
+    plain = orc.muon_step(W0, res[0].M, np.zeros_like(W0), orc.HParams(lr=eta, weight_decay=0.1))
+    assert np.abs(res[0].W - plain.W * (R / np.linalg.norm(plain.W))).max() < 1e-15
+
+
+def test_qk_clip_hand_values():
+    """The QK-Clip listing with tau = 100: a head with S_max = 400 has gamma = 1/4, so its
+    non-rotary q and k rows are halved and its rotary q rows quartered; a head with
+    S_max = 50 is untouched, and so is the shared rotary key."""
+    Wq = np.ones((8, 3))          # heads 0, 1: rows 0-3 / 4-7 (non-rotary q)
+    Wqr = np.ones((4, 3))         # heads 0, 1: rows 0-1 / 2-3 (rotary q)
+    Wk = np.ones((8, 3))          # non-rotary k
+    Wkr = np.ones((2, 3))         # shared rotary k: not in any slice
+    slices = [(0, 0, 4, 0, 0.5), (0, 4, 4, 1, 0.5), (1, 0, 2, 0, 1.0), (1, 2, 2, 1, 1.0),
+              (2, 0, 4, 0, 0.5), (2, 4, 4, 1, 0.5)]
+    q, qr, k, kr = orc.qk_clip([Wq, Wqr, Wk, Wkr], slices, s_max=[400.0, 50.0], tau=100.0)
+    assert np.array_equal(q[:4], np.full((4, 3), 0.5)) and np.array_equal(q[4:], np.ones((4, 3)))
+    assert np.array_equal(qr[:2], np.full((2, 3), 0.25)) and np.array_equal(qr[2:], np.ones((2, 3)))
+    assert np.array_equal(k[:4], np.full((4, 3), 0.5)) and np.array_equal(k[4:], np.ones((4, 3)))
+    assert np.array_equal(kr, Wkr)
+    # after clipping, the head's largest logit q.k scales by gamma^(0.5+0.5) = tau/S_max
+    assert (0.5 * 0.5) * 400.0 == 100.0
+
+
+def test_two_sided_normalisation_rank_one_is_the_sign_pattern():
+    """N(u v^T) = sign(u) sign(v)^T: the row and column factors of a rank-one matrix
+    cancel exactly (eps = 0)."""
+    u = np.array([0.5, -2.0, 3.0, -0.25])
+    v = np.array([1.0, -1e-3, 7.0])
+    got = orc.two_sided_normalise(np.outer(u, v), eps=0.0)
+    assert np.allclose(got, np.outer(np.sign(u), np.sign(v)), rtol=1e-13, atol=0)
+    # scale invariance of the whole step direction: normalisation removes any factor
+    hp = orc.HParams(mode="twosided", scale="none", lr=1.0)
+    W = np.zeros((4, 3))
+    r1 = orc.muon_step(W, np.outer(u, v), np.zeros((4, 3)), hp)
+    r2 = orc.muon_step(W, 1e3 * np.outer(u, v), np.zeros((4, 3)), hp)
+    assert np.allclose(r1.O, r2.O, rtol=1e-5, atol=1e-9)
+    # with eps = 1e-7 the small column (RMS ~7e-5 after normalisation) moves by ~0.14 %
+    assert np.allclose(r1.O, np.outer(np.sign(u), np.sign(v)), rtol=2e-3, atol=0)

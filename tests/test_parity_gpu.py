@@ -98,7 +98,8 @@ STEP_SHAPES = [(17, 33), (33, 17), (128, 256), (256, 128), (200, 700), (320, 512
 
 
 @pytest.mark.parametrize("mode,wd,eq", [("muongs", 0.0, False), ("muon", 0.1, False),
-                                        ("muon", 0.1, True), ("muongs", 0.1, True)])
+                                        ("muon", 0.1, True), ("muongs", 0.1, True),
+                                        ("muonh", 0.0, False), ("muonh", 0.1, True)])
 def test_bf16_step_mixed_shapes_ten_steps(env, mode, wd, eq):
     B, torch = env
     W0 = [H.seeded(r, c, 300 + i, 0.02) for i, (r, c) in enumerate(STEP_SHAPES)]
@@ -149,3 +150,33 @@ def test_degenerate_step_inputs(env):
     gpu = H.run_steps(B, torch, W0, grads, hp, torch.bfloat16)
     assert np.allclose(gpu[0][0][0], (1 - 0.02 * 0.1) * W0[0], rtol=0, atol=1e-7)
     H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs", wd=0.1), H.TOL_BF16)
+
+
+def test_muonh_keeps_the_radius_on_gpu(env):
+    """MuonH: ||W_t|| stays ||W_0|| step after step (fp32 level)."""
+    B, torch = env
+    shapes = [(96, 160), (768, 512)]
+    W0 = [H.seeded(r, c, 40 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded_bf16(r, c, 80 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(4)]
+    gpu = H.run_steps(B, torch, W0, grads, H.gpu_hp(B, mode="muonh", wd=0.1), torch.bfloat16)
+    for i, w in enumerate(W0):
+        R = np.linalg.norm(w.astype(np.float64))
+        for t in range(4):
+            assert abs(np.linalg.norm(gpu[t][0][i]) - R) <= 2e-6 * R
+
+
+def test_two_sided_mode_ten_steps(env):
+    """Two-sided normalisation (no Newton-Schulz, fp32 throughout): 1e-4 against the
+    oracle over 10 steps, scale none, Adam-like learning rate."""
+    B, torch = env
+    shapes = [(17, 33), (128, 256), (300, 64), (512, 320)]
+    W0 = [H.seeded(r, c, 500 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded_bf16(r, c, 600 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(10)]
+    hp = B.hparams(lr=1e-3, weight_decay=0.01, mode="twosided", scale="none")
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.bfloat16)
+    ohp = H.oracle_hp(mode="twosided", wd=0.01, lr=1e-3, scale="none")
+    H.compare_runs(gpu, W0, grads, ohp, H.TOL_FP32, check_stats=False)
+    for t in range(10):
+        assert all(st["equil_axis"] == 3 for st in gpu[t][2])

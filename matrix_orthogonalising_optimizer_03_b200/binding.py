@@ -321,3 +321,56 @@ def qk_clip(slices, s_max, tau: float = 100.0, stream=None):
         raise MuonError(1, "s_max must be a CUDA float32 tensor")
     _check(lib.muon_qk_clip(arr, len(slices), s_max.data_ptr(), s_max.numel(), tau,
                             _stream_ptr(stream)), "muon_qk_clip")
+
+
+class StreamedSteps:
+    """Optimizer steps fed with gradients that arrive from pinned host memory.
+
+    Two device gradient buffers alternate: while step t runs on the compute stream
+    from buffer t % 2, the gradients of step t + 1 are copied into the other buffer
+    on a copy stream, so the host-to-device transfer overlaps the step. Each buffer
+    has its own plan over the same weights and momenta. `step(host_flat)` enqueues
+    the copy of `host_flat` (a pinned tensor holding all gradients back to back, in
+    the order of `params`) and the step that consumes it; the per-matrix statistics
+    of the step are copied back to pinned host memory (`stats_host`).
+    """
+
+    def __init__(self, params, momenta, hp: MuonHParams, grad_dtype=None):
+        torch = _torch()
+        self.params, self.momenta = list(params), list(momenta)
+        dev = self.params[0].device
+        gdt = grad_dtype or torch.bfloat16
+        self.numel = sum(p.numel() for p in self.params)
+        self.bufs, self.plans = [], []
+        for _ in range(2):
+            flat = torch.empty(self.numel, dtype=gdt, device=dev)
+            views, off = [], 0
+            for p in self.params:
+                views.append(flat[off:off + p.numel()].view(p.shape))
+                off += p.numel()
+            self.bufs.append(flat)
+            self.plans.append(Plan(self.params, views, self.momenta, hp))
+        self.stats = new_stats(len(self.params), dev)
+        self.stats_host = torch.empty_like(self.stats, device="cpu").pin_memory()
+        self.copy_stream = torch.cuda.Stream(device=dev)
+        self.copied = [torch.cuda.Event(), torch.cuda.Event()]
+        self.consumed = [torch.cuda.Event(), torch.cuda.Event()]
+        self.t = 0
+
+    def step(self, host_flat, stream=None):
+        torch = _torch()
+        comp = stream or torch.cuda.current_stream()
+        b = self.t % 2
+        with torch.cuda.stream(self.copy_stream):
+            self.copy_stream.wait_event(self.consumed[b])   # buffer b free again
+            self.bufs[b].copy_(host_flat, non_blocking=True)
+            self.copied[b].record(self.copy_stream)
+        comp.wait_event(self.copied[b])
+        self.plans[b].step(stats=self.stats, stream=comp)
+        self.consumed[b].record(comp)
+        self.stats_host.copy_(self.stats, non_blocking=True)
+        self.t += 1
+
+    def close(self):
+        for p in self.plans:
+            p.close()

@@ -211,6 +211,8 @@ __device__ __forceinline__ float ingest_subtile(const ElemArgs& a, const DevMat&
 }
 
 __global__ void __launch_bounds__(kThreads, 8) ingest_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ float tile[kTC][kTR + 1];
   __shared__ double red[1][kThreads / 32];
   const int b = blockIdx.x;
@@ -236,6 +238,8 @@ __device__ __forceinline__ float slab_scale(const ElemArgs& a, int k) {
 
 // ------------------------------------------------------------------ post_reduce
 __global__ void __launch_bounds__(kThreads, 4) post_reduce_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ float tile[kTC][kTR + 1];
   __shared__ double red[3][kThreads / 32];
   __shared__ float colred[2][kTR][kTC + 1];
@@ -346,6 +350,8 @@ __device__ __forceinline__ double block_sum2(double& x, double& y, double (*sh)[
 }
 
 __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ double red[2][kThreads / 32];
   const int k = blockIdx.x;
   const DevMat d = a.mats[k];
@@ -459,6 +465,8 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
 
 // ------------------------------------------------------------------ post_apply
 __global__ void __launch_bounds__(kThreads, 6) post_apply_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
   __shared__ float tile[kTC][kTR + 1];
   const int b = blockIdx.x;
   const int k = find_matrix(a, b);
@@ -506,6 +514,23 @@ __global__ void __launch_bounds__(kThreads, 6) post_apply_kernel(const ElemArgs 
 
 }  // namespace
 
+// Launch with programmatic stream serialisation: the kernel may start while its
+// predecessor finishes and waits for it in griddep_wait().
+template <typename... Args>
+cudaError_t launch_pdl(void (*kern)(Args...), unsigned grid, cudaStream_t s, const ElemArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
   ingest_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
@@ -513,18 +538,15 @@ cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
 }
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
-  post_reduce_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(post_reduce_kernel, a.total_tiles, s, a);
 }
 cudaError_t launch_post_finalize(const ElemArgs& a, cudaStream_t s) {
   if (a.n <= 0) return cudaSuccess;
-  post_finalize_kernel<<<a.n, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(post_finalize_kernel, a.n, s, a);
 }
 cudaError_t launch_post_apply(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
-  post_apply_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(post_apply_kernel, a.total_tiles, s, a);
 }
 
 }  // namespace muon

@@ -104,6 +104,19 @@ __device__ __forceinline__ void named_barrier(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Blocks until the previous kernel in the stream (launched before this one with
+// programmatic stream serialisation) has completed and its memory is visible; a
+// no-op otherwise. Every kernel of a step calls it before touching data written by
+// its predecessor, so the ordering stays transitive along the chain.
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Lets the next kernel of the stream be scheduled while this one finishes.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ CTA pairs (cluster of 2)
 __device__ __forceinline__ uint32_t cluster_cta_rank() {
   uint32_t r;

@@ -42,6 +42,7 @@ def test_full_shape_set_one_step(env, name, run_idx):
     ohp = orc.HParams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
                       equilibrate=run.equilibrate)
     specs = w.matrices()
+    worst = [0.0, 0.0, 0.0]
     for i in picks:
         G = wl.grad(w, specs[i], 0).astype(np.float64)
         r = orc.muon_step(W0[i], G, np.zeros_like(G), ohp)
@@ -50,9 +51,12 @@ def test_full_shape_set_one_step(env, name, run_idx):
         e_w, e_m = H.rel(Wg, r.W), H.rel(Mg, r.M)
         e_dw = H.rel(W0[i] - Wg, W0[i] - r.W)
         assert e_w <= H.TOL_BF16 and e_m <= H.TOL_BF16 and e_dw <= H.TOL_BF16, (i, e_w, e_m, e_dw)
+        worst = [max(worst[0], e_w), max(worst[1], e_m), max(worst[2], e_dw)]
         assert abs(st[i]["w_norm"] - np.linalg.norm(W0[i])) <= 1e-5 * np.linalg.norm(W0[i])
         if run.equilibrate:
             assert st[i]["equil_axis"] in (1, 2)
+    print(f"\nFULLSIZE {name} run {run_idx}: max rel err W {worst[0]:.2e} M {worst[1]:.2e} "
+          f"dW {worst[2]:.2e} over {len(picks)} sampled matrices")
     plan.close()
     del Ws, Gs, Ms
     torch.cuda.empty_cache()

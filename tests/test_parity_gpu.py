@@ -90,6 +90,8 @@ def test_single_128x256_fp32_ten_steps(env, mode):
     hp = H.gpu_hp(B, mode=mode, wd=0.1, ns_fp32=True)
     gpu = H.run_steps(B, torch, W0, grads, hp, torch.float32)
     worst = H.compare_runs(gpu, W0, grads, H.oracle_hp(mode=mode, wd=0.1), H.TOL_FP32)
+    print(f"\nSINGLE {mode}: max rel err over 10 steps W {worst['W']:.2e} M {worst['M']:.2e} "
+          f"dW {worst['dW']:.2e}")
     assert worst["dW"] <= H.TOL_FP32
 
 

@@ -336,6 +336,95 @@ __global__ void __launch_bounds__(kThreads, 4) post_reduce_kernel(const ElemArgs
   }
 }
 
+// ------------------------------------------------------------------ post_reduce (plain)
+// Without equilibration only the three per-matrix sums are needed. For each 64-column
+// band of the super-tile the block handles two 32-row sub-tiles at a time and issues
+// all their loads (W and the slab, 96 bytes per thread) before any arithmetic; tall
+// matrices transpose both slab tiles through shared memory with one barrier pair.
+// The 1/(||U||+eps) slab scale multiplies the finished sums, not every element.
+constexpr int kRedGroup = 2;  // sub-tile rows in flight per thread
+
+template <bool XF32>
+__global__ void __launch_bounds__(kThreads, 4) post_reduce_plain_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ float tile[kRedGroup][kTC][kTR + 1];
+  __shared__ double red[3][kThreads / 32];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
+  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const bool vec = (d.flags & MAT_VEC_OK) != 0;
+  const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  float ww = 0.f, wo = 0.f, oo = 0.f;
+  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
+    const int c0 = C0 + bj * kTC;
+    for (int g0 = 0; g0 < kSubR && R0 + g0 * kTR < d.rows; g0 += kRedGroup) {
+      float w[kRedGroup][8], o[kRedGroup][8];
+      // loads: W in the storage frame; the slab in the storage frame (wide) or as
+      // 64 x 32 tiles of O^T (tall: slab rows = storage columns)
+#pragma unroll
+      for (int q = 0; q < kRedGroup; ++q) {
+        const int r0 = R0 + (g0 + q) * kTR;
+        const int r = r0 + lr, c = c0 + lc;
+        const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+        if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w[q]);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[q][e] = 0.f;
+        }
+        int64_t off;
+        int v2;
+        if (!tall) {
+          off = (int64_t)r * s.ldx + c;
+          v2 = valid;
+        } else {
+          const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
+          off = (int64_t)sr * s.ldx + sc;
+          v2 = (sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
+        }
+        if (v2 > 0) load8_slab(s.xf, XF32, off, v2, o[q]);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[q][e] = 0.f;
+        }
+      }
+      if (tall) {  // block-uniform
+#pragma unroll
+        for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tile[q][threadIdx.x >> 2][(threadIdx.x & 3) * 8 + e] = o[q][e];
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[q][e] = tile[q][lc + e][lr];
+        __syncthreads();  // the tiles are reused by the next group
+      }
+#pragma unroll
+      for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {  // elements outside the matrix are 0 on both sides
+          ww = fmaf(w[q][e], w[q][e], ww);
+          wo = fmaf(w[q][e], o[q][e], wo);
+          oo = fmaf(o[q][e], o[q][e], oo);
+        }
+    }
+  }
+  const double xs = slab_scale(a, k);
+  double acc[3] = {ww, wo * xs, oo * xs * xs};
+  block_sum<3>(acc, red);
+  if (threadIdx.x == 0) {
+    atomicAdd(&a.scal[k].w2, acc[0]);
+    atomicAdd(&a.scal[k].wo, acc[1]);
+    atomicAdd(&a.scal[k].o2, acc[2]);
+  }
+}
+
 // ------------------------------------------------------------------ post_finalize
 __device__ __forceinline__ double block_sum2(double& x, double& y, double (*sh)[kThreads / 32]) {
   double v[2] = {x, y};
@@ -464,10 +553,14 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
 }
 
 // ------------------------------------------------------------------ post_apply
-__global__ void __launch_bounds__(kThreads, 6) post_apply_kernel(const ElemArgs a) {
+// Same walk as the plain reduction: per 64-column band, two 32-row sub-tiles at a time
+// with all loads issued before the arithmetic and, for tall matrices, one shared-memory
+// transpose of the two slab tiles.
+template <bool XF32>
+__global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs a) {
   griddep_launch_dependents();
   griddep_wait();
-  __shared__ float tile[kTC][kTR + 1];
+  __shared__ float tile[kRedGroup][kTC][kTR + 1];
   const int b = blockIdx.x;
   const int k = find_matrix(a, b);
   const DevMat d = a.mats[k];
@@ -477,37 +570,79 @@ __global__ void __launch_bounds__(kThreads, 6) post_apply_kernel(const ElemArgs 
   const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
+  const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  const bool ns_only = a.ns_only != 0;
   const float xs = slab_scale(a, k);
   MatCoef cf;
-  if (!a.ns_only) cf = a.coef[k];
-  for (int bi = 0; bi < kSubR && R0 + bi * kTR < d.rows; ++bi) {
-    for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
-      const int r0 = R0 + bi * kTR, c0 = C0 + bj * kTC;
-      const int r = r0 + lr, c = c0 + lc;
-      const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
-      float o[8];
-      load_o_tile(a, d, s, r0, c0, tile, o);
-      if (valid <= 0) continue;
-      if (a.ns_only) {
+  cf.cw = cf.co = 0.f;
+  cf.axis = 0;
+  if (!ns_only) cf = a.coef[k];
+  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
+    const int c0 = C0 + bj * kTC;
+    const int c = c0 + lc;
+    for (int g0 = 0; g0 < kSubR && R0 + g0 * kTR < d.rows; g0 += kRedGroup) {
+      float w[kRedGroup][8], o[kRedGroup][8];
+      int valid[kRedGroup];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] *= xs;
-        if (d.flags & MAT_G_BF16)
-          store8_bf16(reinterpret_cast<uint16_t*>(d.W) + (int64_t)r * d.ld_w + c, vec, valid, o);
-        else
-          store8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, o);
-        continue;
-      }
-      float w[8];
-      float* wp = d.W + (int64_t)r * d.ld_w + c;
-      load8_f32(wp, vec, valid, w);
-      const float rowf = (cf.axis & 1) ? a.eq_o2[s.eq_off + r] : 1.f;
+      for (int q = 0; q < kRedGroup; ++q) {
+        const int r0 = R0 + (g0 + q) * kTR;
+        const int r = r0 + lr;
+        valid[q] = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+        if (!ns_only && valid[q] > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid[q], w[q]);
+        else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float f = xs * rowf;
-        if ((cf.axis & 2) && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
-        w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
+          for (int e = 0; e < 8; ++e) w[q][e] = 0.f;
+        }
+        int64_t off;
+        int v2;
+        if (!tall) {
+          off = (int64_t)r * s.ldx + c;
+          v2 = valid[q];
+        } else {
+          const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
+          off = (int64_t)sr * s.ldx + sc;
+          v2 = (sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
+        }
+        if (v2 > 0) load8_slab(s.xf, XF32, off, v2, o[q]);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[q][e] = 0.f;
+        }
       }
-      store8_f32(wp, vec, valid, w);
+      if (tall) {  // block-uniform
+#pragma unroll
+        for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tile[q][threadIdx.x >> 2][(threadIdx.x & 3) * 8 + e] = o[q][e];
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[q][e] = tile[q][lc + e][lr];
+        __syncthreads();  // the tiles are reused by the next group
+      }
+#pragma unroll
+      for (int q = 0; q < kRedGroup; ++q) {
+        if (valid[q] <= 0) continue;
+        const int r = R0 + (g0 + q) * kTR + lr;
+        if (ns_only) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[q][e] *= xs;
+          if (d.flags & MAT_G_BF16)
+            store8_bf16(reinterpret_cast<uint16_t*>(d.W) + (int64_t)r * d.ld_w + c, vec, valid[q], o[q]);
+          else
+            store8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid[q], o[q]);
+          continue;
+        }
+        const float rowf = (cf.axis & 1) ? a.eq_o2[s.eq_off + r] : 1.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float f = xs * rowf;
+          if ((cf.axis & 2) && e < valid[q]) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+          w[q][e] = fmaf(cf.cw, w[q][e], cf.co * f * o[q][e]);
+        }
+        store8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid[q], w[q]);
+      }
     }
   }
 }
@@ -538,7 +673,9 @@ cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
 }
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
-  return launch_pdl(post_reduce_kernel, a.total_tiles, s, a);
+  if (a.equilibrate) return launch_pdl(post_reduce_kernel, a.total_tiles, s, a);
+  return a.x_fp32 ? launch_pdl(post_reduce_plain_kernel<true>, a.total_tiles, s, a)
+                  : launch_pdl(post_reduce_plain_kernel<false>, a.total_tiles, s, a);
 }
 cudaError_t launch_post_finalize(const ElemArgs& a, cudaStream_t s) {
   if (a.n <= 0) return cudaSuccess;
@@ -546,7 +683,8 @@ cudaError_t launch_post_finalize(const ElemArgs& a, cudaStream_t s) {
 }
 cudaError_t launch_post_apply(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
-  return launch_pdl(post_apply_kernel, a.total_tiles, s, a);
+  return a.x_fp32 ? launch_pdl(post_apply_kernel<true>, a.total_tiles, s, a)
+                  : launch_pdl(post_apply_kernel<false>, a.total_tiles, s, a);
 }
 
 }  // namespace muon

@@ -7,6 +7,8 @@ with weights, momenta and gradients resident in HBM. Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt160m]
   python bench.py --impl reference ...   # the float64 CPU oracle on host cores
+  python bench.py --impl torch ...       # the same step in eager PyTorch on the GPU
+                                         # (cuBLAS bf16 batched matmuls), for comparison
 
 Multi-GPU (torchrun, one process per GPU): the matrices of a shape set are
 independent, so each rank steps its own copy of the shape set with no collective
@@ -36,7 +38,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference", "torch"])
     ap.add_argument("--workload", default="gpt160m")
     ap.add_argument("--run", type=int, default=0,
                     help="which hyper-parameter setting of the workload (e.g. gpt400m: 0 MuonGS, 1 Muon+wd)")
@@ -208,6 +210,92 @@ def run_reference(args, rank: int, world: int):
     return 0
 
 
+# ------------------------------------------------------------------ eager PyTorch arm
+def run_torch(args, rank: int, world: int, local: int):
+    """The same optimizer step written as eager PyTorch on the GPU, the usual way to run
+    Muon: per shape class one batched tensor, momentum and Nesterov by in-place ops,
+    the quintic Newton-Schulz iteration with bf16 batched matmuls (cuBLAS), the
+    Moonlight scale, the MuonGS projection and the update. No libmuon code runs."""
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    w = wl.WORKLOADS[args.workload]
+    run = w.runs[args.run]
+    if run.equilibrate or run.mode not in ("muon", "muongs") or w.ns_fp32:
+        if rank == 0:
+            print(json.dumps({"impl": "torch", "unavailable": "the eager arm covers bf16 Muon and "
+                              "MuonGS without equilibration"}), flush=True)
+        return 0
+    specs = w.matrices()
+    Ws, G_src = wl.device_inputs(w, dev, seed=rank)
+    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    classes = {}
+    for s, W, G in zip(specs, Ws, G_src):
+        classes.setdefault((s.rows, s.cols), []).append((W, G))
+    batches = []
+    for (r, c), lst in classes.items():
+        W = torch.stack([x[0] for x in lst])
+        G = torch.stack([x[1] for x in lst]).to(gdt)
+        batches.append((W, G, torch.zeros_like(W), r > c, 0.2 * max(r, c) ** 0.5))
+    del Ws, G_src
+    a, b, c = 3.4445, -4.7750, 2.0315
+    mu, lr, wd, eps = w.momentum, w.lr, run.weight_decay, 1e-7
+
+    def step():
+        for W, G, M, tall, scale in batches:
+            M.mul_(mu).add_(G)
+            U = torch.add(G, M, alpha=mu)
+            X = (U / (U.norm(dim=(1, 2), keepdim=True) + eps)).to(torch.bfloat16)
+            if tall:
+                X = X.mT
+            for _ in range(5):
+                A = torch.bmm(X, X.mT)
+                Bm = torch.baddbmm(A, A, A, beta=b, alpha=c)
+                X = torch.baddbmm(X, Bm, X, beta=a, alpha=1.0)
+            O = (X.mT if tall else X).float() * scale
+            cw = torch.full((W.shape[0], 1, 1), 1.0 - lr * wd, device=W.device)
+            if run.mode == "muongs":
+                cw = cw + lr * (W * O).sum(dim=(1, 2), keepdim=True) / (
+                    W * W).sum(dim=(1, 2), keepdim=True).clamp_min(1e-30)
+            W.mul_(cw).add_(O, alpha=-lr)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = rank_max(e0.elapsed_time(e1), world, dev)
+    if rank == 0:
+        value = throughput(args.steps, world, ms)
+        print(json.dumps({
+            "metric": "muon_steps_per_s", "value": value, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "impl": "torch",
+            "config": {"workload": w.name, "matrices": w.n_matrices, "params": w.n_params,
+                       "mode": run.mode, "weight_decay": run.weight_decay,
+                       "ns_path": "torch.bmm / baddbmm bf16 (cuBLAS)",
+                       "parallelism": f"replica x{world}"}}), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 # ------------------------------------------------------------------ multi-rank timing
 def rank_max(x: float, world: int, device="cpu") -> float:
     """The maximum of x over all ranks of the default process group (x itself at
@@ -235,6 +323,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.impl == "torch":
+        return run_torch(args, rank, world, local)
 
     import numpy as np
     import torch

@@ -38,6 +38,9 @@ struct ClassMaps {
   CUtensorMap s64;      // S slab, 64 x 64 boxes (mirror blocks below the diagonal)
   CUtensorMap p128;     // P' slab, 64 x 128 boxes
   CUtensorMap p64;      // P' slab, 64 x 64 boxes
+  CUtensorMap x32[2];   // output boxes of one epilogue warp: 64 x 32
+  CUtensorMap s32;
+  CUtensorMap p32;
 };
 
 }  // namespace
@@ -385,7 +388,10 @@ muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t str
       for (int b = 0; b < 2; ++b) {
         ok = ok && encode_slab_map_bf16(&cm.x128[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 128);
         ok = ok && encode_slab_map_bf16(&cm.x64[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 64);
+        ok = ok && encode_slab_map_bf16(&cm.x32[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 32);
       }
+      ok = ok && encode_slab_map_bf16(&cm.s32, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 32);
+      ok = ok && encode_slab_map_bf16(&cm.p32, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 32);
       ok = ok && encode_slab_map_bf16(&cm.s128, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 128);
       ok = ok && encode_slab_map_bf16(&cm.s64, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 64);
       ok = ok && encode_slab_map_bf16(&cm.p128, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 128);
@@ -618,20 +624,21 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
               if (phase == PH_GRAM) {
                 P.ta[c] = P.ta_t[c] = cm.x128[it % 2];
                 P.tb[c] = P.tb_t[c] = cm.x128[it % 2];
-                P.tc[c] = P.td[c] = cm.s128;
+                P.tc[c] = cm.s128;
+                P.td[c] = cm.s32;
               } else if (phase == PH_POLY) {
                 P.ta[c] = cm.s128;
                 P.ta_t[c] = cm.s64;
                 P.tb[c] = cm.s128;
                 P.tb_t[c] = cm.s64;
                 P.tc[c] = cm.s128;
-                P.td[c] = cm.p128;
+                P.td[c] = cm.p32;
               } else {
                 P.ta[c] = cm.p128;
                 P.ta_t[c] = cm.p64;
                 P.tb[c] = P.tb_t[c] = cm.x64[it % 2];
                 P.tc[c] = cm.x128[it % 2];
-                P.td[c] = cm.x128[(it + 1) % 2];
+                P.td[c] = cm.x32[(it + 1) % 2];
               }
             }
             a.tile_base[cn] = tiles;

@@ -27,10 +27,11 @@
 //              stages (no multicast in any form).
 //   warp 1     TMEM allocator and MMA issuer (one thread), double-buffered fp32
 //              accumulator in TMEM.
-//   warps 2-9  epilogue: two warps per TMEM lane quarter, each taking half of the
-//              columns; tcgen05.ld, fused scale / axpy, bf16 tile staged in swizzled
-//              shared memory and written with TMA bulk stores (which clip ragged
-//              edges). POLY's C tile (S) arrives by TMA one tile ahead.
+//   warps 2-9  epilogue: two warps per TMEM lane quarter, each taking every other
+//              64-column chunk; tcgen05.ld, fused scale / polynomial, and per warp a
+//              32 x 64 bf16 box staged in swizzled shared memory and written with the
+//              warp's own TMA store (which clips ragged edges), with no barrier between
+//              the warps. POLY's C tile (S) arrives by TMA one tile ahead.
 // Two variants:
 //   single CTA   tile 128 x BN (BN = 128 for GRAM / POLY, 256 for APPLY),
 //                tcgen05.mma.cta_group::1, M = 128.
@@ -56,6 +57,7 @@ namespace {
 constexpr int BM = 128, BK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kThreadsTc = 64 + 32 * kEpiWarps;  // 320
+constexpr int kWarpBoxBytes = 32 * 128;           // one 32-row x 64-column bf16 output box
 
 template <int BN, int PHASE, bool PAIR>
 struct TcCfg {
@@ -66,7 +68,11 @@ struct TcCfg {
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = kBRows * BK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStagingBytes = kHasC ? BM * kNCol * 2 : 2 * BM * 64 * 2;  // C tile, or 2 x 16 KB
+  // epilogue: each warp stores 32 x 64 boxes; it takes every other 64-column chunk
+  static constexpr int kChunksPerWarp = kNCol / 128;
+  static constexpr int kEpiBufs = (PAIR && kChunksPerWarp >= 2) ? 2 : 1;  // per-warp box buffers
+  static constexpr int kStagingBytes =
+      kHasC ? BM * kNCol * 2 : kEpiWarps * kEpiBufs * kWarpBoxBytes;  // C tile, or per-warp boxes
   static constexpr int kBudget = 224 * 1024;
   static constexpr int kFit = (kBudget - kStagingBytes) / kStageBytes;
   static constexpr int kStages = kFit > 8 ? 8 : kFit;
@@ -78,7 +84,6 @@ struct TcCfg {
   static constexpr int kMmaN = PAIR ? 256 : BN;
   static constexpr int kTileM = PAIR ? 256 : 128;          // output tile (cluster) rows
   static constexpr int kTileN = PAIR ? 256 : BN;           // output tile columns
-  static constexpr int kRounds = kHasC ? 1 : kNCol / 64;   // output rounds (64 columns each)
   static_assert(kStages >= 3, "pipeline too shallow");
 };
 
@@ -333,11 +338,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2-9)
+    // Each warp owns the 32 accumulator rows of its TMEM lane quarter and every other
+    // 64-column chunk of the tile. It stages a chunk as a 32 x 64 bf16 box in its own
+    // 128B-swizzled buffer (POLY: in place, over the C tile) and stores the box with
+    // its own TMA store, so the warps never wait for one another inside a tile. POLY
+    // synchronises the eight warps once per tile, before the next C tile may land.
     const int ew = warp - 2;
     const int quad = warp & 3;           // the TMEM lane quarter this warp may access
-    const int grp = ew >> 2;             // which half of each 128-column round
+    const int grp = ew >> 2;             // chunks grp, grp + 2, ...
     const int r = quad * 32 + lane;      // tile row of this thread within the CTA
     const bool leader = ew == 0 && lane == 0;
+    uint8_t* wbuf = stg + ew * (C::kEpiBufs * kWarpBoxBytes);  // GRAM / APPLY box buffers
+    int nstore = 0;                                           // boxes this warp has staged
     bool c_pending = false;
     if (HAS_C && leader && unit < total) {
       const TileJob j = decode(p, unit, SYM);
@@ -348,9 +360,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
                     j.ti * C::kTileM + rank * 128, j.mat);
       c_pending = true;
     }
-    // All epilogue warps walk the same tiles and execute every named barrier, also
-    // after a failed wait (they then skip the work): no warp is ever left waiting at
-    // a barrier.
+    // All epilogue warps walk the same tiles and, in POLY, execute every named
+    // barrier, also after a failed wait (they then skip the work): no warp is ever
+    // left waiting at a barrier.
     int it = 0;
     bool ok = true;
     for (int t = unit; t < total; t += nunits, ++it) {
@@ -371,59 +383,24 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
       const int ncols = PHASE == PH_APPLY ? k.n : m;
       const int row0 = j.ti * C::kTileM + rank * 128;   // this CTA's first output row
       const int col0 = j.tj * C::kTileN;                 // this CTA's first output column
-      float scale = 1.f;
       if (ok) {
         if (leader) c_pending = false;
         tc_fence_after();
+        float scale = 1.f;
         if (PHASE != PH_POLY && p.first_iter) {
           const double inv = 1.0 / (sqrt(p.scal[k.first + j.mat].u2) + (double)p.eps);
           scale = static_cast<float>(PHASE == PH_GRAM ? inv * inv : inv);
         }
-      }
-      // Output rounds. POLY writes D over its C tile and stores it whole after the
-      // last round; GRAM / APPLY stage 64 columns per round in two alternating 16 KB
-      // buffers, so a round's store overlaps the next round's math.
 #pragma unroll 1
-      for (int rr = 0; rr < C::kRounds; ++rr) {
-        if (ok) {
-#pragma unroll 1
-          for (int ci = 0; ci < (HAS_C ? C::kNCol / 64 : 1); ++ci) {
-            const int ch = HAS_C ? 2 * ci + grp : 2 * rr + grp;   // 32-column accumulator chunk
-            uint32_t v[32];
-            tmem_ld32(tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                          static_cast<uint32_t>(ab * C::kNCol + ch * 32),
-                      v);
-            tmem_wait_ld();
-            // the element of this row on the global diagonal, as a column of this chunk
-            const int dcol = (row0 + r) - (col0 + ch * 32);
-            uint8_t* buf = HAS_C ? stg : stg + (rr & 1) * (BM * 128);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const uint32_t off = HAS_C ? sw128_off(r, ch * 32 + q4 * 8)
-                                         : sw128_off(r, grp * 32 + q4 * 8);
-              uint4 cw = make_uint4(0, 0, 0, 0);
-              if (HAS_C) cw = *reinterpret_cast<const uint4*>(buf + off);
-              const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
-              uint32_t pk[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int i0 = q4 * 8 + 2 * e;
-                float a0 = __uint_as_float(v[i0]), a1 = __uint_as_float(v[i0 + 1]);
-                if (PHASE == PH_POLY) {
-                  a0 = fmaf(p.b, __uint_as_float(cwv[e] << 16), p.c * a0);
-                  a1 = fmaf(p.b, __uint_as_float(cwv[e] & 0xFFFF0000u), p.c * a1);
-                  if (i0 == dcol) a0 += p.a;
-                  if (i0 + 1 == dcol) a1 += p.a;
-                } else {
-                  a0 *= scale;
-                  a1 *= scale;
-                }
-                pk[e] = pack_bf16x2(a0, a1);
-              }
-              *reinterpret_cast<uint4*>(buf + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-          }
-          if (rr == C::kRounds - 1) {
+        for (int ci = 0; ci < C::kChunksPerWarp; ++ci) {
+          const int c64 = 2 * ci + grp;  // 64-column chunk of the tile
+          uint32_t v[2][32];
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                 static_cast<uint32_t>(ab * C::kNCol + c64 * 64);
+          tmem_ld32(taddr, v[0]);
+          tmem_ld32(taddr + 32, v[1]);
+          tmem_wait_ld();
+          if (ci == C::kChunksPerWarp - 1) {
             // this warp has read its share of the accumulator: free it for the MMA
             tc_fence_before();
             __syncwarp();
@@ -432,44 +409,71 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
               else mbar_arrive_cluster(peer_addr(&tempty[ab], 0));
             }
           }
-          fence_proxy_async_smem();
-        }
-        named_barrier(1, kEpiWarps * 32);
-        if (leader && ok) {
+          uint8_t* box;
           if (HAS_C) {
-            if (row0 < m) {
-#pragma unroll
-              for (int b = 0; b < C::kNCol / 64; ++b)
-                if (col0 + b * 64 < ncols)
-                  tma_store_3d(&P.td[j.c], stg + b * (BM * 128), col0 + b * 64, row0, j.mat);
-            }
-            tma_store_commit();
-            tma_store_wait_read();  // the C / D buffer is free again
-            const int tn = t + nunits;
-            if (tn < total) {
-              const TileJob jn = decode(p, tn, SYM);
-              mbar_expect_tx(cfull, C::kStagingBytes);
-#pragma unroll
-              for (int b = 0; b < C::kNCol / 64; ++b)
-                tma_load_3d(stg + b * (BM * 128), &P.tc[jn.c], cfull, jn.tj * C::kTileN + b * 64,
-                            jn.ti * C::kTileM + rank * 128, jn.mat);
-              c_pending = true;
-            }
+            box = stg + c64 * (BM * 128) + quad * kWarpBoxBytes;  // this warp's rows of C
           } else {
-            const int x = col0 + rr * 64;
-            if (row0 < m && x < ncols)
-              tma_store_3d(&P.td[j.c], stg + (rr & 1) * (BM * 128), x, row0, j.mat);
-            tma_store_commit();
-            tma_store_wait_read_1();  // the previous round's buffer is free again
+            box = wbuf + (nstore % C::kEpiBufs) * kWarpBoxBytes;
+            if (nstore >= C::kEpiBufs) {  // the store that last read this buffer is done with it
+              if (lane == 0) tma_store_wait_read_n<C::kEpiBufs - 1>();
+              __syncwarp();
+            }
           }
+          // the element of this row on the global diagonal, as a column of this chunk
+          const int dcol = (row0 + r) - (col0 + c64 * 64);
+#pragma unroll
+          for (int q8 = 0; q8 < 8; ++q8) {
+            const uint32_t off = sw128_off(lane, q8 * 8);
+            uint4 cw = make_uint4(0, 0, 0, 0);
+            if (HAS_C) cw = *reinterpret_cast<const uint4*>(box + off);
+            const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i0 = q8 * 8 + 2 * e;
+              float a0 = __uint_as_float(v[i0 >> 5][i0 & 31]);
+              float a1 = __uint_as_float(v[(i0 + 1) >> 5][(i0 + 1) & 31]);
+              if (PHASE == PH_POLY) {
+                a0 = fmaf(p.b, __uint_as_float(cwv[e] << 16), p.c * a0);
+                a1 = fmaf(p.b, __uint_as_float(cwv[e] & 0xFFFF0000u), p.c * a1);
+                if (i0 == dcol) a0 += p.a;
+                if (i0 + 1 == dcol) a1 += p.a;
+              } else {
+                a0 *= scale;
+                a1 *= scale;
+              }
+              pk[e] = pack_bf16x2(a0, a1);
+            }
+            *reinterpret_cast<uint4*>(box + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int x = col0 + c64 * 64, y = row0 + quad * 32;
+            if (x < ncols && y < m) tma_store_3d(&P.td[j.c], box, x, y, j.mat);
+            tma_store_commit();
+          }
+          ++nstore;
         }
+      }
+      if (HAS_C) {
+        // every warp's boxes have been read out of the tile; then the next C lands
+        if (lane == 0) tma_store_wait_read();
         named_barrier(1, kEpiWarps * 32);
+        const int tn = t + nunits;
+        if (leader && ok && tn < total) {
+          const TileJob jn = decode(p, tn, SYM);
+          mbar_expect_tx(cfull, C::kStagingBytes);
+#pragma unroll
+          for (int b = 0; b < C::kNCol / 64; ++b)
+            tma_load_3d(stg + b * (BM * 128), &P.tc[jn.c], cfull, jn.tj * C::kTileN + b * 64,
+                        jn.ti * C::kTileM + rank * 128, jn.mat);
+          c_pending = true;
+        }
       }
     }
-    if (leader) {
-      tma_store_wait_all();
-      if (c_pending) mbar_wait(cfull, it & 1, nullptr);  // a C tile still landing
-    }
+    if (lane == 0) tma_store_wait_all();
+    if (leader && c_pending) mbar_wait(cfull, it & 1, nullptr);  // a C tile still landing
   }
 
   __syncthreads();

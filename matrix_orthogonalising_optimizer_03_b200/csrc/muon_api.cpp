@@ -33,11 +33,11 @@ int64_t round_up64(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 
 struct ClassMaps {
   CUtensorMap x128[2];  // X slabs, 64 x 128 boxes (K-major operand, output)
-  CUtensorMap x64[2];   // X slabs, 64 x 64 boxes (MN-major operand of APPLY)
+  CUtensorMap xmn[2];   // X slabs, chunk view (MN-major operand of APPLY)
   CUtensorMap s128;     // S slab, 64 x 128 boxes
-  CUtensorMap s64;      // S slab, 64 x 64 boxes (mirror blocks below the diagonal)
+  CUtensorMap smir;     // S slab, chunk view (mirror blocks below the diagonal)
   CUtensorMap p128;     // P' slab, 64 x 128 boxes
-  CUtensorMap p64;      // P' slab, 64 x 64 boxes
+  CUtensorMap pmir;     // P' slab, chunk view
   CUtensorMap x32[2];   // output boxes of one epilogue warp: 64 x 32
   CUtensorMap s32;
   CUtensorMap p32;
@@ -387,15 +387,16 @@ muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t str
       bool ok = true;
       for (int b = 0; b < 2; ++b) {
         ok = ok && encode_slab_map_bf16(&cm.x128[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 128);
-        ok = ok && encode_slab_map_bf16(&cm.x64[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 64);
+        ok = ok && encode_chunk_map_bf16(&cm.xmn[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx,
+                                         ci.m % kPairTile == 0 ? 2 : tc_block_n(PH_APPLY) / 64);
         ok = ok && encode_slab_map_bf16(&cm.x32[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 32);
       }
       ok = ok && encode_slab_map_bf16(&cm.s32, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 32);
       ok = ok && encode_slab_map_bf16(&cm.p32, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 32);
       ok = ok && encode_slab_map_bf16(&cm.s128, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 128);
-      ok = ok && encode_slab_map_bf16(&cm.s64, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 64);
+      ok = ok && encode_chunk_map_bf16(&cm.smir, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 2);
       ok = ok && encode_slab_map_bf16(&cm.p128, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 128);
-      ok = ok && encode_slab_map_bf16(&cm.p64, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 64);
+      ok = ok && encode_chunk_map_bf16(&cm.pmir, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 2);
       if (!ok) return MUON_ERR_CUDA;
     }
   }
@@ -628,15 +629,15 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
                 P.td[c] = cm.s32;
               } else if (phase == PH_POLY) {
                 P.ta[c] = cm.s128;
-                P.ta_t[c] = cm.s64;
+                P.ta_t[c] = cm.smir;
                 P.tb[c] = cm.s128;
-                P.tb_t[c] = cm.s64;
+                P.tb_t[c] = cm.smir;
                 P.tc[c] = cm.s128;
                 P.td[c] = cm.p32;
               } else {
                 P.ta[c] = cm.p128;
-                P.ta_t[c] = cm.p64;
-                P.tb[c] = P.tb_t[c] = cm.x64[it % 2];
+                P.ta_t[c] = cm.pmir;
+                P.tb[c] = P.tb_t[c] = cm.xmn[it % 2];
                 P.tc[c] = cm.x128[it % 2];
                 P.td[c] = cm.x32[(it + 1) % 2];
               }

@@ -235,14 +235,14 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
         P.tc[0] = P.td[0];
       } else if (phase == PH_POLY) {
         ok = encode_slab_map_bf16(&P.ta[0], k.s, m, m, 1, lds, 64, 128) &&
-             encode_slab_map_bf16(&P.ta_t[0], k.s, m, m, 1, lds, 64, 64) &&
+             encode_chunk_map_bf16(&P.ta_t[0], k.s, m, m, 1, lds, 2) &&
              encode_slab_map_bf16(&P.td[0], k.p, m, m, 1, lds, 64, 32);
         P.tb[0] = P.tc[0] = P.ta[0];
         P.tb_t[0] = P.ta_t[0];
       } else {
         ok = encode_slab_map_bf16(&P.ta[0], k.p, m, m, 1, lds, 64, 128) &&
-             encode_slab_map_bf16(&P.ta_t[0], k.p, m, m, 1, lds, 64, 64) &&
-             encode_slab_map_bf16(&P.tb[0], x_in, n, m, 1, ldx, 64, 64) &&
+             encode_chunk_map_bf16(&P.ta_t[0], k.p, m, m, 1, lds, 2) &&
+             encode_chunk_map_bf16(&P.tb[0], x_in, n, m, 1, ldx, bn / 64) &&
              encode_slab_map_bf16(&P.tc[0], x_in, n, m, 1, ldx, 64, 128) &&
              encode_slab_map_bf16(&P.td[0], k.x_out, n, m, 1, ldx, 64, 32);
         P.tb_t[0] = P.tb[0];

@@ -19,8 +19,10 @@
 // Symmetric storage: S and P' are symmetric, so only their 128 x 128 blocks on or
 // above the block diagonal are computed and stored. A consumer that needs a block
 // below the diagonal (rows in block i, columns in block k < i) loads its mirror
-// block (k, i) with 64 x 64 TMA boxes and hands it to tcgen05.mma as an MN-major
-// operand (the transpose is free in the instruction descriptor).
+// block (k, i) and hands it to tcgen05.mma as an MN-major operand (the transpose is
+// free in the instruction descriptor). MN-major blocks (these mirrors and APPLY's X)
+// come in one TMA box of a 4-D view of the slab, [matrix][64-column chunk][row][64],
+// which lands chunk after chunk in the MN-major layout.
 //
 // Kernel structure (persistent, one CTA per SM, 320 threads):
 //   warp 0     TMA producer: a STAGES-deep ring of 128B-swizzled shared-memory
@@ -131,8 +133,9 @@ __device__ __forceinline__ bool below_diag(bool sym_operand, int tile_row0, int 
   return sym_operand && (kb * BK) / G < tile_row0 / G;
 }
 
-// Loads the 128 x 64 block of a K-major operand, or its mirror as two 64 x 64
-// boxes (MN-major layout, 8 KB apart) when it lies below the diagonal.
+// Loads the 128 x 64 block of a K-major operand, or, when it lies below the
+// diagonal, its mirror as one box of the chunk view (two 64 x 64 chunks, 8 KB apart:
+// the MN-major layout).
 template <bool PAIR>
 __device__ __forceinline__ void load_k_block(uint8_t* dst, const CUtensorMap* mk,
                                              const CUtensorMap* mt, uint64_t* bar, int row0,
@@ -141,11 +144,8 @@ __device__ __forceinline__ void load_k_block(uint8_t* dst, const CUtensorMap* mk
     if (PAIR) tma_load_3d_pair(dst, mk, bar, kb * BK, row0, mat);
     else tma_load_3d(dst, mk, bar, kb * BK, row0, mat);
   } else {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (PAIR) tma_load_3d_pair(dst + h * (64 * BK * 2), mt, bar, row0 + h * 64, kb * BK, mat);
-      else tma_load_3d(dst + h * (64 * BK * 2), mt, bar, row0 + h * 64, kb * BK, mat);
-    }
+    if (PAIR) tma_load_4d_pair(dst, mt, bar, 0, kb * BK, row0 / 64, mat);
+    else tma_load_4d(dst, mt, bar, 0, kb * BK, row0 / 64, mat);
   }
 }
 
@@ -241,12 +241,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           if (!B_MN) {
             load_k_block<PAIR>(sb, &P.tb[j.c], &P.tb_t[j.c], &full[s], b_row0, kb, j.mat,
                                below_diag(B_SYM, j.tj * C::kTileN, kb, C::kTileN));
-          } else {
-#pragma unroll
-            for (int h = 0; h < C::kBRows / 64; ++h) {
-              if (PAIR) tma_load_3d_pair(sb + h * (64 * BK * 2), &P.tb[j.c], &full[s], b_row0 + h * 64, kb * BK, j.mat);
-              else tma_load_3d(sb + h * (64 * BK * 2), &P.tb[j.c], &full[s], b_row0 + h * 64, kb * BK, j.mat);
-            }
+          } else {  // X rows kb*BK.., columns b_row0.. in kBRows/64 chunks, one box
+            if (PAIR) tma_load_4d_pair(sb, &P.tb[j.c], &full[s], 0, kb * BK, b_row0 / 64, j.mat);
+            else tma_load_4d(sb, &P.tb[j.c], &full[s], 0, kb * BK, b_row0 / 64, j.mat);
           }
           ++q;
         }
@@ -562,6 +559,32 @@ bool encode_slab_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_chunk_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int64_t rows,
+                           int64_t count, int64_t ld, int box_chunks) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  if (encode == nullptr) {
+    cudaDriverEntryPointQueryResult qr;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
+            cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess || fn == nullptr)
+      return false;
+    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  if (ld % 64 != 0) return false;  // every chunk lies inside a slab row
+  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>((inner + 63) / 64), static_cast<cuuint64_t>(count)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(ld * 2), 128,
+                           static_cast<cuuint64_t>(rows * ld * 2)};
+  cuuint32_t box[4] = {64, 64, static_cast<cuuint32_t>(box_chunks), 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = encode(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -35,5 +35,12 @@ constexpr int kPairTile = 256;
 
 bool encode_slab_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int64_t rows,
                           int64_t count, int64_t ld, int box_inner, int box_rows);
+// 4-D view of the same slab as [count][column chunk of 64][rows][64] (innermost
+// first: 64 columns, rows, chunks, matrices) with a box of 64 rows x `box_chunks`
+// chunks, 128B swizzle: one load brings a block in the MN-major operand layout
+// (chunk after chunk). Columns past `inner` in its last chunk are the slab's padding
+// and are read as stored; they only reach output rows / columns the stores clip.
+bool encode_chunk_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int64_t rows,
+                           int64_t count, int64_t ld, int box_chunks);
 
 }  // namespace muon

@@ -182,3 +182,44 @@ def test_two_sided_mode_ten_steps(env):
     H.compare_runs(gpu, W0, grads, ohp, H.TOL_FP32, check_stats=False)
     for t in range(10):
         assert all(st["equil_axis"] == 3 for st in gpu[t][2])
+
+
+def test_strided_unaligned_views_ten_steps(env):
+    """W, G and M as column slices of wider buffers at odd offsets: ld > cols, rows not
+    16-byte aligned, so the elementwise kernels take their scalar paths. Parity against
+    the oracle over 10 steps, and nothing outside the views is written."""
+    B, torch = env
+    cases = [((200, 300), 333, 1), ((300, 130), 141, 3), ((256, 300), 301, 1),
+             ((300, 256), 259, 2), ((33, 17), 40, 5)]
+    W0 = [H.seeded(r, c, 1100 + i, 0.02) for i, ((r, c), _, _) in enumerate(cases)]
+    grads = [[H.seeded_bf16(r, c, 1200 + 10 * t + i, 1e-3) for i, ((r, c), _, _) in enumerate(cases)]
+             for t in range(10)]
+    bufs_w, bufs_m, bufs_g, Ws, Ms, Gs = [], [], [], [], [], []
+    for i, ((r, c), ld, off) in enumerate(cases):
+        bw = torch.full((r, ld), 7.0, dtype=torch.float32, device="cuda")
+        bm = torch.full((r, ld), -3.0, dtype=torch.float32, device="cuda")
+        bg = torch.zeros((r, ld + 2), dtype=torch.bfloat16, device="cuda")
+        w = bw[:, off:off + c]
+        w.copy_(torch.from_numpy(W0[i]))
+        m = bm[:, off:off + c]
+        m.zero_()
+        bufs_w.append(bw), bufs_m.append(bm), bufs_g.append(bg)
+        Ws.append(w), Ms.append(m), Gs.append(bg[:, off + 1:off + 1 + c])
+    hp = H.gpu_hp(B, mode="muongs", wd=0.1)
+    plan = B.Plan(Ws, Gs, Ms, hp)
+    stats = B.new_stats(len(Ws))
+    gpu = []
+    for gl in grads:
+        for g_dev, g in zip(Gs, gl):
+            g_dev.copy_(torch.from_numpy(np.ascontiguousarray(g, dtype=np.float32)))
+        plan.step(stats=stats)
+        torch.cuda.synchronize()
+        gpu.append(([w.double().cpu().numpy() for w in Ws], [m.double().cpu().numpy() for m in Ms],
+                    B.decode_stats(stats)))
+    assert plan.query_device_status() == 0
+    plan.close()
+    H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs", wd=0.1), H.TOL_BF16)
+    for i, ((r, c), ld, off) in enumerate(cases):
+        for buf, fill in ((bufs_w[i], 7.0), (bufs_m[i], -3.0)):
+            outside = torch.cat([buf[:, :off], buf[:, off + c:]], dim=1)
+            assert bool((outside == fill).all()), (i, fill)

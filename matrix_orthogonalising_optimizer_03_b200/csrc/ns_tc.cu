@@ -26,7 +26,7 @@
 //
 // Kernel structure (persistent, one CTA per SM, 320 threads):
 //   warp 0     TMA producer: a STAGES-deep ring of 128B-swizzled shared-memory
-//              stages (no multicast in any form).
+//              stages; every load lands in one CTA's own shared memory.
 //   warp 1     TMEM allocator and MMA issuer (one thread), double-buffered fp32
 //              accumulator in TMEM.
 //   warps 2-9  epilogue: two warps per TMEM lane quarter, each taking every other

@@ -57,7 +57,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 __device__ __forceinline__ void tma_prefetch(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
-// 3-D tiled load (no multicast) of one box into shared memory; completion is
+// 3-D tiled load of one box into this CTA's shared memory; completion is
 // signalled on `bar` as transaction bytes.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y, int z) {
@@ -68,8 +68,8 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// 4-D tiled load (no multicast): used for 64-column-chunk views of a slab, whose box
-// lands in shared memory chunk after chunk (the MN-major operand layout).
+// 4-D tiled load into this CTA's shared memory: used for 64-column-chunk views of a
+// slab, whose box lands chunk after chunk (the MN-major operand layout).
 __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y, int z, int w) {
   asm volatile(

@@ -49,6 +49,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "muon_internal.h"
 #include "ns_tc.h"
 #include "ptx.cuh"
@@ -485,13 +487,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
 template <int BN, int PHASE, bool PAIR>
 cudaError_t launch_tc(const TcParams& P, int grid, cudaStream_t s) {
   using C = TcCfg<BN, PHASE, PAIR>;
-  static bool attr_set = false;
+  // the shared-memory opt-in is a per-device attribute: set it once on each device
+  static std::atomic<uint64_t> attr_devices{0};
   auto kern = ns_tc_kernel<BN, PHASE, PAIR>;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit == 0 || !(attr_devices.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    attr_devices.fetch_or(bit, std::memory_order_acq_rel);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
@@ -540,18 +546,25 @@ cudaError_t launch_ns_phase_tc(const TcParams& P, int num_sms, cudaStream_t s) {
 
 // Encodes a 3-D bf16 tensor map over a slab [count][rows][ld] with a
 // box_inner x box_rows box (128B swizzle). Returns false on failure.
+// The driver's cuTensorMapEncodeTiled, looked up once (thread-safe static init);
+// null when the driver does not provide it.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+    cudaDriverEntryPointQueryResult qr;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) !=
+            cudaSuccess ||
+        qr != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
 bool encode_slab_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int64_t rows,
                           int64_t count, int64_t ld, int box_inner, int box_rows) {
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  if (encode == nullptr) {
-    cudaDriverEntryPointQueryResult qr;
-    void* fn = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
-            cudaSuccess ||
-        qr != cudaDriverEntryPointSuccess || fn == nullptr)
-      return false;
-    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(count)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * 2),
@@ -567,16 +580,8 @@ bool encode_slab_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int
 
 bool encode_chunk_map_bf16(CUtensorMap* out, const void* base, int64_t inner, int64_t rows,
                            int64_t count, int64_t ld, int box_chunks) {
-  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
-  if (encode == nullptr) {
-    cudaDriverEntryPointQueryResult qr;
-    void* fn = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
-            cudaSuccess ||
-        qr != cudaDriverEntryPointSuccess || fn == nullptr)
-      return false;
-    encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  }
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return false;
   if (ld % 64 != 0) return false;  // every chunk lies inside a slab row
   cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>((inner + 63) / 64), static_cast<cuuint64_t>(count)};

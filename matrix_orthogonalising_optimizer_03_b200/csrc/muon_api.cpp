@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -333,29 +334,26 @@ muon_plan_s* make_ns_plan(const muon_ns_matrix_t* mats, int n, const muon_hparam
   return p;
 }
 
-struct DeviceInfo {
-  bool checked = false;
-  bool ok = false;
-  int num_sms = 0;
-};
-DeviceInfo g_dev[kMaxDevices];
+// Per-device facts, queried once. `info` packs them (bit 31: queried, bit 30: sm_100,
+// low bits: SM count) so that a thread reads either nothing or the whole record.
+std::atomic<uint32_t> g_dev_info[kMaxDevices];
 
 muon_status_t current_device(int* dev, int* num_sms) {
   if (cudaGetDevice(dev) != cudaSuccess) return MUON_ERR_CUDA;
   if (*dev < 0 || *dev >= kMaxDevices) return MUON_ERR_UNSUPPORTED;
-  DeviceInfo& di = g_dev[*dev];
-  if (!di.checked) {
+  uint32_t info = g_dev_info[*dev].load(std::memory_order_acquire);
+  if (!(info & 0x80000000u)) {
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess)
       return MUON_ERR_CUDA;
-    di.ok = (major == 10 && minor == 0);
-    di.num_sms = sms;
-    di.checked = true;
+    info = 0x80000000u | ((major == 10 && minor == 0) ? 0x40000000u : 0u) |
+           (static_cast<uint32_t>(sms) & 0xFFFFu);
+    g_dev_info[*dev].store(info, std::memory_order_release);
   }
-  if (!di.ok) return MUON_ERR_UNSUPPORTED;
-  *num_sms = di.num_sms;
+  if (!(info & 0x40000000u)) return MUON_ERR_UNSUPPORTED;
+  *num_sms = static_cast<int>(info & 0xFFFFu);
   return MUON_OK;
 }
 

@@ -20,6 +20,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include <cstdint>
 #include <cstring>
 
@@ -52,8 +54,9 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[muon::kNoAllocS
 namespace muon {
 namespace {
 
-void* g_scratch_addr[kNoAllocMaxDevices];  // device address of g_noalloc_scratch, per device
-int g_num_sms[kNoAllocMaxDevices];
+// Per device: the device address of g_noalloc_scratch (published last) and the SM count.
+std::atomic<void*> g_scratch_addr[kNoAllocMaxDevices];
+std::atomic<int> g_num_sms[kNoAllocMaxDevices];
 
 // Writes the one-matrix descriptor tables and clears the scalars and status words.
 __global__ void noalloc_setup_kernel(unsigned char* base, DevMat d, DevSlab s, int32_t tiles,
@@ -74,7 +77,8 @@ muon_status_t scratch_for_current_device(unsigned char** out, int* num_sms) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return MUON_ERR_UNSUPPORTED;
-  if (g_scratch_addr[dev] == nullptr) {
+  void* addr = g_scratch_addr[dev].load(std::memory_order_acquire);
+  if (addr == nullptr) {
     int major = 0, minor = 0, sms = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -84,11 +88,12 @@ muon_status_t scratch_for_current_device(unsigned char** out, int* num_sms) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
       return MUON_ERR_CUDA;
-    g_num_sms[dev] = sms;
-    g_scratch_addr[dev] = p;
+    g_num_sms[dev].store(sms, std::memory_order_relaxed);
+    g_scratch_addr[dev].store(p, std::memory_order_release);
+    addr = p;
   }
-  *out = static_cast<unsigned char*>(g_scratch_addr[dev]);
-  *num_sms = g_num_sms[dev];
+  *out = static_cast<unsigned char*>(addr);
+  *num_sms = g_num_sms[dev].load(std::memory_order_relaxed);
   return MUON_OK;
 }
 

@@ -171,6 +171,18 @@ def matrix_array(params, grads, momenta):
     return arr
 
 
+def _device_of(tensors):
+    """The CUDA device of the first tensor (the library runs on the current device, so
+    every call switches to the device that holds its matrices); None for empty lists."""
+    return tensors[0].device if len(tensors) else None
+
+
+def _on(device):
+    """Context that makes `device` current for one library call."""
+    import contextlib
+    return _torch().cuda.device(device) if device is not None else contextlib.nullcontext()
+
+
 def _stream_ptr(stream) -> Optional[int]:
     torch = _torch()
     if stream is None:
@@ -224,8 +236,10 @@ def step_batched(params, grads, momenta, hp: MuonHParams, workspace=None, stats=
         if n and size == 0:
             _check(lib.muon_validate(arr, n, ctypes.byref(hp)), "muon_validate")
         workspace = new_workspace(size, params[0].device if n else "cuda")
-    _check(lib.muon_step_batched(arr, n, ctypes.byref(hp), workspace.data_ptr(), workspace.numel(),
-                                 _stats_ptr(stats), _stream_ptr(stream)), "muon_step_batched")
+    with _on(_device_of(params)):
+        _check(lib.muon_step_batched(arr, n, ctypes.byref(hp), workspace.data_ptr(),
+                                     workspace.numel(), _stats_ptr(stats), _stream_ptr(stream)),
+               "muon_step_batched")
     return workspace
 
 
@@ -243,19 +257,24 @@ class Plan:
                "muon_plan_create")
         self._plan = h
         self.workspace_bytes = int(self._lib.muon_plan_workspace_size(h))
-        dev = params[0].device if self.n else "cuda"
-        self.workspace = workspace if workspace is not None else new_workspace(self.workspace_bytes, dev)
+        self.device = _device_of(params)
+        self.workspace = (workspace if workspace is not None
+                          else new_workspace(self.workspace_bytes, self.device or "cuda"))
 
     def set_hparams(self, hp: MuonHParams):
         _check(self._lib.muon_plan_set_hparams(self._plan, ctypes.byref(hp)), "muon_plan_set_hparams")
         self.hp = hp
 
     def step(self, stats=None, stream=None):
-        _check(self._lib.muon_plan_step(self._plan, self.workspace.data_ptr(), self.workspace.numel(),
-                                        _stats_ptr(stats), _stream_ptr(stream)), "muon_plan_step")
+        with _on(self.device):
+            _check(self._lib.muon_plan_step(self._plan, self.workspace.data_ptr(),
+                                            self.workspace.numel(), _stats_ptr(stats),
+                                            _stream_ptr(stream)), "muon_plan_step")
 
     def query_device_status(self, stream=None) -> int:
-        return int(self._lib.muon_query_device_status(self.workspace.data_ptr(), _stream_ptr(stream)))
+        with _on(self.device):
+            return int(self._lib.muon_query_device_status(self.workspace.data_ptr(),
+                                                          _stream_ptr(stream)))
 
     def close(self):
         if getattr(self, "_plan", None):
@@ -285,9 +304,10 @@ def newton_schulz(xs, outs, hp: MuonHParams, workspace=None, stream=None):
     if workspace is None:
         size = lib.muon_ns_workspace_size(arr, n, ctypes.byref(hp))
         workspace = new_workspace(size, xs[0].device if n else "cuda")
-    _check(lib.muon_newton_schulz_batched(arr, n, ctypes.byref(hp), workspace.data_ptr(),
-                                          workspace.numel(), _stream_ptr(stream)),
-           "muon_newton_schulz_batched")
+    with _on(_device_of(xs)):
+        _check(lib.muon_newton_schulz_batched(arr, n, ctypes.byref(hp), workspace.data_ptr(),
+                                              workspace.numel(), _stream_ptr(stream)),
+               "muon_newton_schulz_batched")
     return workspace
 
 
@@ -302,9 +322,10 @@ def newton_schulz_noalloc(x, o, hp: MuonHParams, status=None, stream=None):
         raise MuonError(3, "X and O must have the same dtype and shape")
     m = MuonNSMatrix(x.data_ptr(), o.data_ptr(), x.size(0), x.size(1), max(x.stride(0), x.size(1)),
                      max(o.stride(0), o.size(1)), _dtype_code(x), 0)
-    _check(lib.muon_newton_schulz_noalloc(ctypes.byref(m), ctypes.byref(hp),
-                                          status.data_ptr() if status is not None else None,
-                                          _stream_ptr(stream)), "muon_newton_schulz_noalloc")
+    with _on(x.device):
+        _check(lib.muon_newton_schulz_noalloc(ctypes.byref(m), ctypes.byref(hp),
+                                              status.data_ptr() if status is not None else None,
+                                              _stream_ptr(stream)), "muon_newton_schulz_noalloc")
 
 
 def qk_clip(slices, s_max, tau: float = 100.0, stream=None):
@@ -319,8 +340,9 @@ def qk_clip(slices, s_max, tau: float = 100.0, stream=None):
         arr[i] = MuonQkSlice(w.data_ptr(), r0, nr, w.size(1), max(w.stride(0), w.size(1)), h, pw)
     if s_max.dtype != _torch().float32 or not s_max.is_cuda:
         raise MuonError(1, "s_max must be a CUDA float32 tensor")
-    _check(lib.muon_qk_clip(arr, len(slices), s_max.data_ptr(), s_max.numel(), tau,
-                            _stream_ptr(stream)), "muon_qk_clip")
+    with _on(s_max.device):
+        _check(lib.muon_qk_clip(arr, len(slices), s_max.data_ptr(), s_max.numel(), tau,
+                                _stream_ptr(stream)), "muon_qk_clip")
 
 
 class StreamedSteps:

@@ -223,3 +223,57 @@ def test_strided_unaligned_views_ten_steps(env):
         for buf, fill in ((bufs_w[i], 7.0), (bufs_m[i], -3.0)):
             outside = torch.cat([buf[:, :off], buf[:, off + c:]], dim=1)
             assert bool((outside == fill).all()), (i, fill)
+
+
+@pytest.mark.parametrize("g_fp32,scale,nesterov,ns_steps", [(True, "keller", False, 5),
+                                                            (False, "none", True, 3),
+                                                            (True, "moonlight", True, 5)])
+def test_bf16_path_option_combinations(env, g_fp32, scale, nesterov, ns_steps):
+    """The bf16 tensor-core path with fp32 gradients, the Keller / no scale rules, plain
+    momentum (U = M) and a non-default iteration count, against the oracle over 4 steps."""
+    B, torch = env
+    shapes = [(96, 160), (256, 384), (384, 256), (70, 70)]
+    W0 = [H.seeded(r, c, 1300 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    gen = H.seeded if g_fp32 else H.seeded_bf16
+    grads = [[gen(r, c, 1400 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(4)]
+    hp = H.gpu_hp(B, mode="muongs", wd=0.05, scale=scale, nesterov=nesterov, ns_steps=ns_steps)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.float32 if g_fp32 else torch.bfloat16)
+    ohp = H.oracle_hp(mode="muongs", wd=0.05, scale=scale, nesterov=nesterov, ns_steps=ns_steps)
+    H.compare_runs(gpu, W0, grads, ohp, H.TOL_BF16)
+
+
+def test_plan_hparams_change_between_steps(env):
+    """muon_plan_set_hparams between steps: two Muon steps at lr 0.02, then two MuonGS
+    steps at lr 0.01 with decay and 4 Newton-Schulz iterations (the result moves to the
+    other slab), on the same plan, momenta carried over. W_t and dW_t per step."""
+    B, torch = env
+    shapes = [(128, 256), (512, 256)]
+    W0 = [H.seeded(r, c, 1500 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded_bf16(r, c, 1600 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(4)]
+    Ws = [torch.tensor(w, device="cuda") for w in W0]
+    Ms = [torch.zeros_like(w) for w in Ws]
+    Gs = [torch.empty(w.shape, dtype=torch.bfloat16, device="cuda") for w in Ws]
+    plan = B.Plan(Ws, Gs, Ms, H.gpu_hp(B, mode="muon", lr=0.02))
+    W_orc = [w.astype(np.float64) for w in W0]
+    M_orc = [np.zeros_like(w) for w in W_orc]
+    for t in range(4):
+        if t == 2:
+            plan.set_hparams(H.gpu_hp(B, mode="muongs", lr=0.01, wd=0.1, ns_steps=4))
+        ohp = (H.oracle_hp(mode="muon", lr=0.02) if t < 2
+               else H.oracle_hp(mode="muongs", lr=0.01, wd=0.1, ns_steps=4))
+        W_prev_gpu = [w.double().cpu().numpy() for w in Ws]
+        W_prev_orc = [w.copy() for w in W_orc]
+        for g_dev, g in zip(Gs, grads[t]):
+            g_dev.copy_(torch.from_numpy(np.ascontiguousarray(g, dtype=np.float32)))
+        plan.step()
+        torch.cuda.synchronize()
+        for i in range(len(shapes)):
+            r = orc.muon_step(W_orc[i], grads[t][i].astype(np.float64), M_orc[i], ohp)
+            W_orc[i], M_orc[i] = r.W, r.M
+            Wg = Ws[i].double().cpu().numpy()
+            assert H.rel(Wg, W_orc[i]) <= H.TOL_BF16, (t, i)
+            assert H.rel(W_prev_gpu[i] - Wg, W_prev_orc[i] - W_orc[i]) <= H.TOL_BF16, (t, i)
+    assert plan.query_device_status() == 0
+    plan.close()

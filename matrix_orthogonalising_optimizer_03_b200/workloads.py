@@ -195,7 +195,7 @@ def device_inputs(w: Workload, device, seed: int = 0, exact=(), step: int = 0):
     return Ws, Gs
 
 
-def sample_indices(w: Workload, extra: int = 3, seed: int = 7) -> List[int]:
+def sample_indices(w: Workload, extra: int = 8, seed: int = 7) -> List[int]:
     """One matrix per shape class (its first) plus `extra` seeded picks: the matrices a
     full-size parity check compares with the oracle one by one."""
     first = {}

@@ -3,16 +3,18 @@
 //   ingest        a1 momentum M = mu*M + G, a2 Nesterov U = G + mu*M, ||U||_F^2,
 //                 and U written to the Newton-Schulz slab in the oriented frame
 //                 (transposed through shared memory for tall matrices).
-//   post_reduce   ||W||^2, <W,O>, ||O||^2 and, for equilibration, per-row and
-//                 per-column sums of O^2 and W*O (storage frame).
+//   post_reduce   ||W||^2, <W,O>, ||O||^2 (post_reduce_plain_kernel); with
+//                 equilibration also per-row and per-column sums of O^2 and W*O in the
+//                 storage frame (post_reduce_eq_kernel).
 //   post_finalize one block per matrix: equilibration axis and factors (a6),
 //                 scale (a7), GS coefficient (a8), statistics, update coefficients.
 //   post_apply    a9: W <- cw*W + co*D*O (or, Newton-Schulz only, O out).
 //
 // Work unit: a 128 x 256 super-tile of the matrix in its storage frame per
 // 256-thread block, walked as 4 x 4 sub-tiles of 32 x 64 (8 consecutive columns
-// per thread, 128-bit accesses when aligned). The super-tile of each block is
-// found by binary search over a per-matrix tile prefix. Per-matrix sums use one
+// per thread, 128-bit accesses when aligned; the plain reduction and post_apply
+// take two 32-row sub-tiles at a time). The super-tile of each block is found by
+// binary search over a per-matrix tile prefix. Per-matrix sums use one
 // atomic per block; the equilibration row / column sums are reduced inside the
 // block (shuffles for rows, a shared-memory transpose for columns) and use one
 // atomic per row and per column of the super-tile.
@@ -236,8 +238,10 @@ __device__ __forceinline__ float slab_scale(const ElemArgs& a, int k) {
   return static_cast<float>(1.0 / (sqrt(a.scal[k].u2) + (double)a.eps));
 }
 
-// ------------------------------------------------------------------ post_reduce
-__global__ void __launch_bounds__(kThreads, 4) post_reduce_kernel(const ElemArgs a) {
+// ------------------------------------------------------------------ post_reduce (equilibration)
+// Equilibration and the two-sided mode: the three per-matrix sums plus the per-row and
+// per-column sums of O^2 and W*O.
+__global__ void __launch_bounds__(kThreads, 4) post_reduce_eq_kernel(const ElemArgs a) {
   griddep_launch_dependents();
   griddep_wait();
   __shared__ float tile[kTC][kTR + 1];
@@ -673,7 +677,7 @@ cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
 }
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
-  if (a.equilibrate) return launch_pdl(post_reduce_kernel, a.total_tiles, s, a);
+  if (a.equilibrate) return launch_pdl(post_reduce_eq_kernel, a.total_tiles, s, a);
   return a.x_fp32 ? launch_pdl(post_reduce_plain_kernel<true>, a.total_tiles, s, a)
                   : launch_pdl(post_reduce_plain_kernel<false>, a.total_tiles, s, a);
 }

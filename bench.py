@@ -492,8 +492,9 @@ def roofline(prof, w, peaks, peak_src, workload, region_ms: float):
     flops = v["flops"] / v["launches"]
     achieved = flops / per_launch_s / 1e12
     if w.ns_fp32:
+        alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
         return {"bound": "alu", "kernel": name, "achieved": achieved, "unit": "TFLOP/s",
-                "peak": 148 * 128 * 2 * 1.965e9 / 1e12, "frac": None, "traffic": None,
+                "peak": alu_peak, "frac": achieved / alu_peak, "traffic": None,
                 "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x 1965 MHz"}
     # a kernel inside a timed region of a second or more runs under the power cap:
     # compare it with the sustained figure, a shorter region with the burst figure

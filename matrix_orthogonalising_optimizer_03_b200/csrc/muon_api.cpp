@@ -74,12 +74,30 @@ struct muon_plan_s {
   bool prof = false;
   std::vector<ProfRec> recs;
   std::vector<cudaEvent_t> event_pool;
+  // A cached plan replays its step as a CUDA graph (one launch instead of ~20) while
+  // the workspace, the stats pointer, the device and the hyper-parameters stay the
+  // same. The first step runs eagerly (lazy per-device setup); the next one is captured
+  // on a private stream; a failed capture leaves the plan eager for good.
+  bool use_graph = false;
+  bool graph_ok = true;
+  int eager_steps = 0;
+  cudaGraphExec_t graph_exec = nullptr;
+  void* graph_ws = nullptr;
+  muon_stats_t* graph_stats = nullptr;
+  int graph_dev = -1;
+  cudaStream_t cap_stream = nullptr;
+  void drop_graph() {
+    if (graph_exec != nullptr) cudaGraphExecDestroy(graph_exec);
+    graph_exec = nullptr;
+  }
   ~muon_plan_s() {
     for (const ProfRec& r : recs) {
       cudaEventDestroy(r.a);
       cudaEventDestroy(r.b);
     }
     for (cudaEvent_t e : event_pool) cudaEventDestroy(e);
+    drop_graph();
+    if (cap_stream != nullptr) cudaStreamDestroy(cap_stream);
   }
 };
 
@@ -501,19 +519,10 @@ double elem_bytes(const muon_plan_s* p, int kind) {
   return total;
 }
 
-muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* stats,
-                       cudaStream_t stream) {
-  if (p->n == 0) return MUON_OK;
-  if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < p->ws_bytes)
-    return MUON_ERR_WORKSPACE;
-  int dev = 0, num_sms = 0;
-  muon_status_t st = current_device(&dev, &num_sms);
-  if (st != MUON_OK) return st;
-  p->num_sms = num_sms;
-  if (p->ws_cached != ws || p->dev_cached != dev) {
-    st = bind_workspace(p, ws, dev, stream);
-    if (st != MUON_OK) return st;
-  }
+// Enqueues one step (memsets and kernel launches only, so it can be captured) on
+// `stream`, for a plan already bound to workspace `ws` on the current device.
+muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int num_sms,
+                           cudaStream_t stream) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int n = p->n;
   const muon_hparams_t& hp = p->hp;
@@ -669,6 +678,67 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
   return MUON_OK;
 }
 
+// Captures one step of a bound plan into a CUDA graph on the plan's private stream.
+muon_status_t capture_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int dev, int num_sms) {
+  p->drop_graph();
+  if (p->cap_stream == nullptr &&
+      cudaStreamCreateWithFlags(&p->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  if (cudaStreamBeginCapture(p->cap_stream, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  const muon_status_t st = enqueue_step(p, ws, stats, num_sms, p->cap_stream);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(p->cap_stream, &graph);
+  if (st != MUON_OK || e != cudaSuccess || graph == nullptr) {
+    if (graph != nullptr) cudaGraphDestroy(graph);
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  const cudaError_t ei = cudaGraphInstantiate(&exec, graph, 0);
+  cudaGraphDestroy(graph);
+  if (ei != cudaSuccess || exec == nullptr) {
+    cudaGetLastError();
+    return MUON_ERR_CUDA;
+  }
+  p->graph_exec = exec;
+  p->graph_ws = ws;
+  p->graph_stats = stats;
+  p->graph_dev = dev;
+  return MUON_OK;
+}
+
+muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* stats,
+                       cudaStream_t stream) {
+  if (p->n == 0) return MUON_OK;
+  if (ws == nullptr || reinterpret_cast<uintptr_t>(ws) % kAlign != 0 || ws_bytes < p->ws_bytes)
+    return MUON_ERR_WORKSPACE;
+  int dev = 0, num_sms = 0;
+  muon_status_t st = current_device(&dev, &num_sms);
+  if (st != MUON_OK) return st;
+  p->num_sms = num_sms;
+  if (p->ws_cached != ws || p->dev_cached != dev) {
+    p->drop_graph();
+    st = bind_workspace(p, ws, dev, stream);
+    if (st != MUON_OK) return st;
+  }
+  if (p->use_graph && p->graph_ok && !p->prof) {
+    const bool same = p->graph_exec != nullptr && p->graph_ws == ws && p->graph_stats == stats &&
+                      p->graph_dev == dev;
+    if (!same && p->eager_steps > 0 && capture_step(p, ws, stats, dev, num_sms) != MUON_OK)
+      p->graph_ok = false;  // stay eager
+    if (p->graph_ok && p->graph_exec != nullptr && p->graph_ws == ws && p->graph_stats == stats &&
+        p->graph_dev == dev)
+      return cudaGraphLaunch(p->graph_exec, stream) == cudaSuccess ? MUON_OK : MUON_ERR_CUDA;
+  }
+  ++p->eager_steps;
+  return enqueue_step(p, ws, stats, num_sms, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -741,6 +811,7 @@ muon_status_t muon_plan_create(const muon_matrix_t* mats, int n, const muon_hpar
   if (st != MUON_OK) return st;
   muon_plan_s* p = make_step_plan(mats, n, hp);
   if (p == nullptr) return MUON_ERR_INVALID_ARG;
+  p->use_graph = true;
   *out = p;
   return MUON_OK;
 }
@@ -758,6 +829,7 @@ muon_status_t muon_plan_set_hparams(muon_plan_t plan, const muon_hparams_t* hp) 
   const bool parity_changed = (steps % 2) != (plan->ns_steps % 2);
   plan->hp = *hp;
   plan->ns_steps = steps;
+  plan->drop_graph();                             // the captured launches hold the old values
   if (parity_changed) plan->ws_cached = nullptr;  // the result slab moved: re-upload
   return MUON_OK;
 }

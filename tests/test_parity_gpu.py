@@ -277,3 +277,42 @@ def test_plan_hparams_change_between_steps(env):
             assert H.rel(W_prev_gpu[i] - Wg, W_prev_orc[i] - W_orc[i]) <= H.TOL_BF16, (t, i)
     assert plan.query_device_status() == 0
     plan.close()
+
+
+def test_plan_graph_replay_matches_eager_steps(env):
+    """A cached plan runs its first step eagerly, captures the second into a CUDA graph
+    and replays it afterwards (re-capturing when the stats pointer changes). Four plan
+    steps must equal four one-shot muon_step_batched calls (never graphed) up to the
+    order of the atomic sums."""
+    B, torch = env
+    shapes = [(128, 256), (300, 130), (256, 256)]
+    W0 = [H.seeded(r, c, 1700 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded_bf16(r, c, 1800 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(4)]
+    hp = H.gpu_hp(B, mode="muongs", wd=0.05)
+    runs = []
+    for use_plan in (True, False):
+        Ws = [torch.tensor(w, device="cuda") for w in W0]
+        Ms = [torch.zeros_like(w) for w in Ws]
+        Gs = [torch.empty(w.shape, dtype=torch.bfloat16, device="cuda") for w in Ws]
+        stats = B.new_stats(len(Ws))
+        plan = B.Plan(Ws, Gs, Ms, hp) if use_plan else None
+        for t in range(4):
+            for g_dev, g in zip(Gs, grads[t]):
+                g_dev.copy_(torch.from_numpy(np.ascontiguousarray(g, dtype=np.float32)))
+            st = stats if t != 2 else None          # step 3 has no stats: a new graph
+            if use_plan:
+                plan.step(stats=st)
+            else:
+                B.step_batched(Ws, Gs, Ms, hp, stats=st)
+        torch.cuda.synchronize()
+        if plan is not None:
+            assert plan.query_device_status() == 0
+            plan.close()
+        runs.append(([w.double().cpu().numpy() for w in Ws], [m.double().cpu().numpy() for m in Ms],
+                     B.decode_stats(stats)))
+    for i in range(len(shapes)):
+        assert H.rel(runs[0][0][i], runs[1][0][i]) <= 1e-5, i
+        assert H.rel(runs[0][1][i], runs[1][1][i]) <= 1e-6, i
+        for key in ("w_norm", "o_norm"):
+            assert abs(runs[0][2][i][key] - runs[1][2][i][key]) <= 1e-5 * abs(runs[1][2][i][key]) + 1e-9

@@ -390,7 +390,8 @@ class StreamedSteps:
         comp.wait_event(self.copied[b])
         self.plans[b].step(stats=self.stats, stream=comp)
         self.consumed[b].record(comp)
-        self.stats_host.copy_(self.stats, non_blocking=True)
+        with torch.cuda.stream(comp):   # the read-back follows the step on its stream
+            self.stats_host.copy_(self.stats, non_blocking=True)
         self.t += 1
 
     def close(self):

@@ -179,8 +179,9 @@ def two_sided_normalise(X: np.ndarray, eps: float = 1e-7) -> np.ndarray:
     pages give no formula. Reading: with r_i and c_j the mean squares of row i and
     column j and rho the RMS of X, N_ij = X_ij rho / ((sqrt(r_i) + eps)(sqrt(c_j) + eps)),
     the rank-one (row x column) estimate of the second moment a second-moment
-    optimizer would divide by. A rank-one X = u v^T maps to sign(u) sign(v)^T.
-    PARITY UNPINNED beyond that closed form."""
+    optimizer would divide by. Closed form: a scaled sign matrix X = D_r Z D_c (Z of
+    +-1 entries, D_r, D_c positive diagonal) maps to Z; rank one, X = u v^T, maps to
+    sign(u) sign(v)^T. PARITY UNPINNED beyond that closed form."""
     r = np.mean(X * X, axis=1)
     c = np.mean(X * X, axis=0)
     rho = np.sqrt(np.mean(X * X))

@@ -325,3 +325,20 @@ def test_two_sided_normalisation_rank_one_is_the_sign_pattern():
     assert np.allclose(r1.O, r2.O, rtol=1e-5, atol=1e-9)
     # with eps = 1e-7 the small column (RMS ~7e-5 after normalisation) moves by ~0.14 %
     assert np.allclose(r1.O, np.outer(np.sign(u), np.sign(v)), rtol=2e-3, atol=0)
+
+
+def test_two_sided_normalisation_of_a_scaled_sign_matrix_is_the_sign_matrix():
+    """N(D_r Z D_c) = Z for any +-1 matrix Z (full rank in general) and positive row and
+    column scalings D_r, D_c (eps = 0): the row mean square of X is d_ri^2 mean(d_c^2), the
+    column one d_cj^2 mean(d_r^2), and the RMS sqrt(mean(d_r^2) mean(d_c^2)), so every
+    factor cancels. The rank-one case is Z = sign(u) sign(v)^T."""
+    rng = np.random.default_rng(21)
+    for rows, cols in ((5, 7), (16, 3), (1, 9), (12, 12)):
+        Z = rng.choice([-1.0, 1.0], size=(rows, cols))
+        dr = np.exp(rng.normal(0.0, 1.5, rows))
+        dc = np.exp(rng.normal(0.0, 1.5, cols))
+        X = dr[:, None] * Z * dc[None, :]
+        got = orc.two_sided_normalise(X, eps=0.0)
+        assert np.allclose(got, Z, rtol=1e-12, atol=0), (rows, cols)
+        if rows > 1 and cols > 1:
+            assert np.linalg.matrix_rank(Z) > 1 or rows * cols <= 4

@@ -162,7 +162,8 @@ def equilibrate(O: np.ndarray, eps: float = 1e-7) -> Tuple[np.ndarray, int]:
     std(v)/mean(v); rows are balanced if imbalance(r) >= imbalance(c), else
     columns; each chosen line is rescaled to the global RMS rho = RMS(O):
     O_ij <- O_ij * rho / (r_i + eps) (columns likewise), which keeps ||O||_F.
-    PARITY UNPINNED beyond its invariants.
+    Closed form: a line-scaled sign matrix D_r Z (or Z D_c) picks rows (columns) and maps
+    to RMS(O) * Z. PARITY UNPINNED beyond that closed form and the invariants.
     """
     r = np.sqrt(np.mean(O * O, axis=1))
     c = np.sqrt(np.mean(O * O, axis=0))

@@ -342,3 +342,20 @@ def test_two_sided_normalisation_of_a_scaled_sign_matrix_is_the_sign_matrix():
         assert np.allclose(got, Z, rtol=1e-12, atol=0), (rows, cols)
         if rows > 1 and cols > 1:
             assert np.linalg.matrix_rank(Z) > 1 or rows * cols <= 4
+
+
+def test_equilibration_of_line_scaled_sign_matrices():
+    """O = D_r Z (Z of +-1 entries, D_r positive and not constant): every column has the
+    same RMS, sqrt(mean(d^2)), while the rows do not, so rows are chosen and
+    O_ij <- d_i z_ij rho / d_i = rho z_ij with rho = RMS(O) (eps = 0). The column-scaled
+    O = Z D_c maps to rho Z through the columns. ||O||_F is kept in both cases."""
+    rng = np.random.default_rng(22)
+    for rows, cols in ((6, 9), (9, 6), (10, 10)):
+        Z = rng.choice([-1.0, 1.0], size=(rows, cols))
+        d = np.exp(rng.normal(0.0, 1.0, max(rows, cols)))
+        for O, axis in ((d[:rows, None] * Z, orc.AXIS_ROWS), (Z * d[None, :cols], orc.AXIS_COLS)):
+            rho = np.sqrt(np.mean(O * O))
+            got, ax = orc.equilibrate(O, eps=0.0)
+            assert ax == axis, (rows, cols, axis)
+            assert np.allclose(got, rho * Z, rtol=1e-12, atol=0)
+            assert np.linalg.norm(got) == pytest.approx(np.linalg.norm(O), rel=1e-12)

@@ -230,7 +230,9 @@ MUON_API int muon_plan_profile_read(muon_plan_t plan, muon_profile_entry_t* out,
  * allocator owning all device memory, which must not be bypassed; code that
  * cannot afford the device-wide synchronisation cudaMalloc/cudaFree may imply.
  * Same result as muon_newton_schulz_batched for that one matrix (X in, O out,
- * device pointers, dtype F32 or BF16 for both). Scratch is the library's own
+ * device pointers, dtype F32 or BF16 for both): the arguments are validated by
+ * the same host checks (so they get the same status) and the same kernels and tile
+ * shapes run. Scratch is the library's own
  * 32 MiB static device array, which every GPU that loads the library keeps
  * until exit. A matrix whose scratch needs exceed it is rejected with
  * MUON_ERR_WORKSPACE before anything is enqueued. In bf16 that is 2*(m*ld_n +
@@ -240,8 +242,12 @@ MUON_API int muon_plan_profile_read(muon_plan_t plan, muon_profile_entry_t* out,
  * two host threads) race and must be serialised by the caller. The first call
  * on each device looks up the array's device address (cudaGetSymbolAddress,
  * with that device current), so make it before any stream capture.
- * status_dev: optional device uint32 that receives MUON_ERR_TIMEOUT if a bounded
- * wait inside a kernel gives up (cleared to 0 at the start of the call). */
+ * status_dev: optional uint32 in device memory of the current device (anything
+ * else is rejected with MUON_ERR_INVALID_ARG) that receives MUON_ERR_TIMEOUT if a
+ * bounded wait inside a kernel gives up; it is cleared to 0 at the start of the
+ * call. With status_dev == NULL a timeout is not reported anywhere: the word it
+ * lands in belongs to the shared scratch and the next call clears it, and O may
+ * then hold garbage. Pass a status word whenever the result matters. */
 MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matrix_t* mat,
                                                   const muon_hparams_t* hp, uint32_t* status_dev,
                                                   void* stream);
@@ -274,8 +280,9 @@ MUON_API muon_status_t muon_qk_clip(const muon_qk_slice_t* slices, int n, const 
  * workspace needs only its first 256 bytes. Nothing faults and nothing hangs. */
 MUON_API muon_status_t muon_wait_probe(void* workspace, int64_t limit_cycles, void* stream);
 
-/* Synchronises `stream`, returns the sticky device-side error word of the
- * workspace (MUON_OK or MUON_ERR_TIMEOUT) and clears it. The word is zeroed when
+/* Reads the sticky device-side error word of the workspace (MUON_OK or
+ * MUON_ERR_TIMEOUT) behind the work already enqueued on `stream`, clears it on that
+ * stream, and synchronises `stream` only (no other stream and no device-wide wait). The word is zeroed when
  * a plan first uses a workspace and on every muon_step_batched /
  * muon_newton_schulz_batched call, so after those it reflects that call only. */
 MUON_API muon_status_t muon_query_device_status(void* workspace, void* stream);

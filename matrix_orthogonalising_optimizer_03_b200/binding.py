@@ -199,6 +199,22 @@ def _stats_ptr(stats) -> Optional[int]:
     return stats.data_ptr()
 
 
+def _status_ptr(status) -> Optional[int]:
+    """Device address of a one-word status tensor (int32 or uint32, at least one
+    element, on a CUDA device), or None. Anything else raises before any launch."""
+    if status is None:
+        return None
+    torch = _torch()
+    ok_dtypes = [torch.int32] + ([torch.uint32] if hasattr(torch, "uint32") else [])
+    if not status.is_cuda:
+        raise MuonError(1, "status must be a CUDA tensor")
+    if status.dtype not in ok_dtypes:
+        raise MuonError(1, f"status must be int32 or uint32 (got {status.dtype})")
+    if status.numel() < 1:
+        raise MuonError(1, "status must have at least one element")
+    return status.data_ptr()
+
+
 def new_stats(n: int, device="cuda"):
     """A device buffer for n muon_stats_t (int32 storage; see `decode_stats`)."""
     return _torch().zeros((n, 6), dtype=_torch().int32, device=device)
@@ -316,15 +332,19 @@ def newton_schulz_noalloc(x, o, hp: MuonHParams, status=None, stream=None):
     instead of a workspace (for callers that cannot allocate device memory).
     status: optional CUDA int32/uint32 one-element tensor for the device error word."""
     lib = load()
+    status_ptr = _status_ptr(status)
     _check_2d(x, "X")
     _check_2d(o, "O")
     if x.dtype != o.dtype or tuple(x.shape) != tuple(o.shape):
         raise MuonError(3, "X and O must have the same dtype and shape")
+    if o.device != x.device:
+        raise MuonError(1, "X and O must be on the same device")
+    if status is not None and status.device != x.device:
+        raise MuonError(1, "status must be on the device of X")
     m = MuonNSMatrix(x.data_ptr(), o.data_ptr(), x.size(0), x.size(1), max(x.stride(0), x.size(1)),
                      max(o.stride(0), o.size(1)), _dtype_code(x), 0)
     with _on(x.device):
-        _check(lib.muon_newton_schulz_noalloc(ctypes.byref(m), ctypes.byref(hp),
-                                              status.data_ptr() if status is not None else None,
+        _check(lib.muon_newton_schulz_noalloc(ctypes.byref(m), ctypes.byref(hp), status_ptr,
                                               _stream_ptr(stream)), "muon_newton_schulz_noalloc")
 
 

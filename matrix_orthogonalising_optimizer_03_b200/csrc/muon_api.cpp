@@ -176,7 +176,11 @@ muon_status_t validate_step(const muon_matrix_t* mats, int n, const muon_hparams
   return MUON_OK;
 }
 
-muon_status_t validate_ns(const muon_ns_matrix_t* mats, int n, const muon_hparams_t* hp) {
+}  // namespace
+
+// Host validation of a Newton-Schulz-only list, shared by muon_newton_schulz_batched,
+// muon_ns_workspace_size and muon_newton_schulz_noalloc (declared in muon_internal.h).
+muon_status_t muon::validate_ns(const muon_ns_matrix_t* mats, int n, const muon_hparams_t* hp) {
   if (hp == nullptr || n < 0 || (n > 0 && mats == nullptr)) return MUON_ERR_INVALID_ARG;
   if (!valid_enum_hp(hp)) return MUON_ERR_INVALID_ARG;
   std::vector<Interval> iv;
@@ -196,6 +200,8 @@ muon_status_t validate_ns(const muon_ns_matrix_t* mats, int n, const muon_hparam
   if (any_alias(iv)) return MUON_ERR_ALIAS;
   return MUON_OK;
 }
+
+namespace {
 
 // Groups matrices by oriented shape and lays out the workspace.
 void build_plan(muon_plan_s* p) {
@@ -895,13 +901,16 @@ muon_status_t muon_newton_schulz_batched(const muon_ns_matrix_t* mats, int n,
 
 muon_status_t muon_query_device_status(void* workspace, void* stream) {
   if (workspace == nullptr) return MUON_ERR_INVALID_ARG;
+  // ordered on `stream` only: the read follows the work enqueued there, the clear
+  // is enqueued behind it, and no other stream of the caller is waited for
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t word = 0;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return MUON_ERR_CUDA;
-  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
     return MUON_ERR_CUDA;
-  if (word != 0 && cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return MUON_ERR_CUDA;
-  if (cudaDeviceSynchronize() != cudaSuccess) return MUON_ERR_CUDA;
+  if (word != 0 && (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess ||
+                    cudaStreamSynchronize(s) != cudaSuccess))
+    return MUON_ERR_CUDA;
   return word == 0 ? MUON_OK : static_cast<muon_status_t>(word);
 }
 

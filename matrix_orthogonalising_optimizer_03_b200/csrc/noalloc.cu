@@ -105,25 +105,14 @@ using namespace muon;
 extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matrix_t* mat,
                                                               const muon_hparams_t* hp,
                                                               uint32_t* status_dev, void* stream) {
-  // ---- host validation (nothing is enqueued on error)
-  if (mat == nullptr || hp == nullptr) return MUON_ERR_INVALID_ARG;
-  if (mat->X == nullptr || mat->O == nullptr) return MUON_ERR_INVALID_ARG;
-  if (hp->ns_steps < 0 || hp->ns_steps > 64 || !(hp->eps >= 0.f)) return MUON_ERR_INVALID_ARG;
-  if (hp->flags & ~static_cast<uint32_t>(MUON_NESTEROV | MUON_EQUILIBRATE | MUON_NS_FP32 |
-                                         MUON_WANT_STATS))
-    return MUON_ERR_INVALID_ARG;
+  // ---- host validation (nothing is enqueued on error): the same checks as
+  // muon_newton_schulz_batched, so one set of arguments gets one status from both
+  if (mat == nullptr) return MUON_ERR_INVALID_ARG;
+  muon_status_t st = validate_ns(mat, 1, hp);
+  if (st != MUON_OK) return st;
   const int64_t rows = mat->rows, cols = mat->cols;
-  if (rows < 1 || cols < 1 || rows > (1 << 24) || cols > (1 << 24) ||
-      rows * cols >= (int64_t(1) << 31))
-    return MUON_ERR_SHAPE;
-  if (mat->ld_x < cols || mat->ld_o < cols) return MUON_ERR_SHAPE;
-  if (mat->dtype != MUON_F32 && mat->dtype != MUON_BF16) return MUON_ERR_DTYPE;
   const int esz = mat->dtype == MUON_BF16 ? 2 : 4;
   const uintptr_t xa = reinterpret_cast<uintptr_t>(mat->X), oa = reinterpret_cast<uintptr_t>(mat->O);
-  if (xa % esz || oa % esz) return MUON_ERR_INVALID_ARG;
-  const uintptr_t xe = xa + static_cast<uintptr_t>(((rows - 1) * mat->ld_x + cols) * esz);
-  const uintptr_t oe = oa + static_cast<uintptr_t>(((rows - 1) * mat->ld_o + cols) * esz);
-  if (xa < oe && oa < xe) return MUON_ERR_ALIAS;
 
   const bool fp32 = (hp->flags & MUON_NS_FP32) != 0;
   const int ex = fp32 ? 4 : 2;
@@ -146,8 +135,21 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
 
   unsigned char* base = nullptr;
   int num_sms = 0;
-  muon_status_t st = scratch_for_current_device(&base, &num_sms);
+  st = scratch_for_current_device(&base, &num_sms);
   if (st != MUON_OK) return st;
+  if (status_dev != nullptr) {
+    // the setup kernel stores to it: it must be device memory of the current device
+    int dev = 0;
+    cudaPointerAttributes pa;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MUON_ERR_CUDA;
+    if (cudaPointerGetAttributes(&pa, status_dev) != cudaSuccess) {
+      cudaGetLastError();
+      return MUON_ERR_INVALID_ARG;
+    }
+    if ((pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged) || pa.device != dev ||
+        reinterpret_cast<uintptr_t>(status_dev) % 4 != 0)
+      return MUON_ERR_INVALID_ARG;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* err = status_dev != nullptr ? status_dev : reinterpret_cast<uint32_t*>(base + kOffHeader);
 
@@ -189,10 +191,13 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
   ea.xs_from_u2 = iterate ? 0 : 1;
   if (launch_ingest(ea, s) != cudaSuccess) return MUON_ERR_CUDA;
 
+  // the same kernels and tile shapes the batched path picks for this shape: CTA
+  // pairs with 256 x 256 tiles when m is a multiple of 256, single CTAs otherwise
+  const bool pair = !fp32 && m % kPairTile == 0;
   for (int it = 0; it < hp->ns_steps; ++it) {
     for (int phase = PH_GRAM; phase <= PH_APPLY; ++phase) {
-      const int bm = fp32 ? 64 : tc_block_m();
-      const int bn = fp32 ? 64 : tc_block_n(phase);
+      const int bm = fp32 ? 64 : (pair ? kPairTile : tc_block_m());
+      const int bn = fp32 ? 64 : (pair ? kPairTile : tc_block_n(phase));
       const int bk = fp32 ? 16 : tc_block_k();
       TcParams P;
       std::memset(&P, 0, sizeof(P));
@@ -235,9 +240,9 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
       // S and P' hold only their blocks on or above the diagonal; *_t maps fetch mirrors
       if (phase == PH_GRAM) {
         ok = encode_slab_map_bf16(&P.ta[0], x_in, n, m, 1, ldx, 64, 128) &&
+             encode_slab_map_bf16(&P.tc[0], k.s, m, m, 1, lds, 64, 128) &&
              encode_slab_map_bf16(&P.td[0], k.s, m, m, 1, lds, 64, 32);
         P.ta_t[0] = P.tb[0] = P.tb_t[0] = P.ta[0];
-        P.tc[0] = P.td[0];
       } else if (phase == PH_POLY) {
         ok = encode_slab_map_bf16(&P.ta[0], k.s, m, m, 1, lds, 64, 128) &&
              encode_chunk_map_bf16(&P.ta_t[0], k.s, m, m, 1, lds, 2) &&
@@ -247,13 +252,16 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
       } else {
         ok = encode_slab_map_bf16(&P.ta[0], k.p, m, m, 1, lds, 64, 128) &&
              encode_chunk_map_bf16(&P.ta_t[0], k.p, m, m, 1, lds, 2) &&
-             encode_chunk_map_bf16(&P.tb[0], x_in, n, m, 1, ldx, bn / 64) &&
+             encode_chunk_map_bf16(&P.tb[0], x_in, n, m, 1, ldx,
+                                   pair ? 2 : tc_block_n(PH_APPLY) / 64) &&
              encode_slab_map_bf16(&P.tc[0], x_in, n, m, 1, ldx, 64, 128) &&
              encode_slab_map_bf16(&P.td[0], k.x_out, n, m, 1, ldx, 64, 32);
         P.tb_t[0] = P.tb[0];
       }
       if (!ok) return MUON_ERR_CUDA;
-      if (launch_ns_phase_tc(P, num_sms, s) != cudaSuccess) return MUON_ERR_CUDA;
+      const cudaError_t e = pair ? launch_ns_phase_tc_pair(P, num_sms, s)
+                                 : launch_ns_phase_tc(P, num_sms, s);
+      if (e != cudaSuccess) return MUON_ERR_CUDA;
     }
   }
   if (launch_post_apply(ea, s) != cudaSuccess) return MUON_ERR_CUDA;

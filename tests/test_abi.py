@@ -127,3 +127,74 @@ def test_workspace_size_and_plan_are_host_only(lib):
     hp.flags |= B.MUON_NS_FP32
     assert lib.muon_workspace_size(arr, 4, ctypes.byref(hp)) > ws    # fp32 slabs
     assert lib.muon_workspace_size(arr, 4, None) == 0
+
+
+def _ns(x, o, rows, cols, ldx=None, ldo=None, dtype=1):
+    return B.MuonNSMatrix(x, o, rows, cols, ldx or cols, ldo or cols, dtype, 0)
+
+
+def _ns_arr(m):
+    a = (B.MuonNSMatrix * 1)()
+    a[0] = m
+    return a
+
+
+def test_both_newton_schulz_entry_points_give_the_same_status(lib):
+    """The workspace entry point and the no-alloc entry point validate through one host
+    routine: every bad argument gets the same status from both, before any CUDA call."""
+    def hp_with(**kw):
+        hp = B.MuonHParams()
+        lib.muon_hparams_default(ctypes.byref(hp))
+        for k, v in kw.items():
+            setattr(hp, k, v)
+        return hp
+
+    ok = _ns(FAKE, FAKE + (1 << 30), 64, 96)
+    cases = [
+        (ok, hp_with(eps=float("inf")), 1), (ok, hp_with(eps=float("nan")), 1),
+        (ok, hp_with(eps=-1.0), 1), (ok, hp_with(mode=9), 1), (ok, hp_with(scale=7), 1),
+        (ok, hp_with(flags=0x100), 1), (ok, hp_with(ns_steps=-1), 1), (ok, hp_with(ns_steps=65), 1),
+        (_ns(0, FAKE, 4, 4), hp_with(), 1), (_ns(FAKE, FAKE + (1 << 30), 0, 4), hp_with(), 2),
+        (_ns(FAKE, FAKE + (1 << 30), 4, 8, ldx=4), hp_with(), 2),
+        (_ns(FAKE, FAKE + (1 << 30), 4, 8, dtype=5), hp_with(), 3),
+        (_ns(FAKE, FAKE + 8, 4, 8), hp_with(), 4),                    # O overlaps X
+        (_ns(FAKE + 1, FAKE + (1 << 30), 4, 8), hp_with(), 1),         # misaligned bf16 X
+    ]
+    for m, hp, want in cases:
+        batched = lib.muon_newton_schulz_batched(_ns_arr(m), 1, ctypes.byref(hp), None, 0, None)
+        noalloc = lib.muon_newton_schulz_noalloc(ctypes.byref(m), ctypes.byref(hp), None, None)
+        assert batched == noalloc == want, (want, batched, noalloc)
+    assert lib.muon_newton_schulz_noalloc(None, ctypes.byref(hp_with()), None, None) == 1
+    assert lib.muon_newton_schulz_noalloc(ctypes.byref(ok), None, None, None) == 1
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor where only attributes are inspected."""
+
+    def __init__(self, dtype, numel, device="cuda:0"):
+        import torch
+        self.dtype, self._numel, self.is_cuda = dtype, numel, True
+        self.device = torch.device(device)
+
+    def numel(self):
+        return self._numel
+
+    def data_ptr(self):
+        raise AssertionError("a rejected status tensor must never be dereferenced")
+
+
+def test_noalloc_binding_rejects_bad_status_before_any_launch(lib):
+    """A status word that is not a one-element int32/uint32 CUDA tensor raises MuonError
+    before the library is called (the kernels would otherwise store through it)."""
+    import torch
+    hp = B.hparams()
+    x = torch.zeros(8, 8, dtype=torch.bfloat16)
+    o = torch.zeros(8, 8, dtype=torch.bfloat16)
+    bad = [torch.zeros(1, dtype=torch.int32),               # host memory
+           _FakeCudaTensor(torch.int64, 1),                  # wrong dtype
+           _FakeCudaTensor(torch.float32, 1),
+           _FakeCudaTensor(torch.int32, 0)]                  # empty
+    for status in bad:
+        with pytest.raises(B.MuonError) as e:
+            B.newton_schulz_noalloc(x, o, hp, status=status)
+        assert e.value.status == 1 and "status" in str(e.value)

@@ -1,7 +1,8 @@
 """The accumulated-learning-rate study on the GPU path: C_T = sum_t eta / ||W_t|| from
-the per-step statistics of the plan, against the bounds of "Muon이 weight decay 없이도
-안정적인 이유" (Theorem 4.1, Proposition 4.2) for MuonGS and the MuonW radius bound of
-its section "무엇과 다른가" for decoupled weight decay.
+the per-step statistics of the plan, against the bounds of "MuonGS: Pretraining LLMs
+with Relaxed Weight-Norm Control" (section 전제와 한계: Theorem 4.1, Proposition 4.2)
+for MuonGS and the MuonW radius bound of its section "무엇과 다른가" for decoupled
+weight decay.
 
 The bounds are stated for an update of Frobenius norm at most sqrt(p); the quintic
 Newton-Schulz iteration only approximates the polar factor, so p is replaced by the

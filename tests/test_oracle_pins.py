@@ -219,6 +219,75 @@ def test_muonw_radius_bound():
     assert orc.accumulated_lr([eta] * T, [r.w_norm for r in res]) >= eta * T / R
 
 
+def test_bound_helpers_hand_values():
+    """The three bound helpers of the MuonGS page at hand-computed points.
+    Theorem 4.1: (2/(p eta)) (sqrt(r0^2 + p eta^2 T) - r0);
+    Proposition 4.2: eta T / sqrt(r0^2 + 2 p eta^2 T);
+    무엇과 다른가: R_lambda = max(r0, sqrt(p) / lambda)."""
+    # r0 = 0, p = 4, eta = 1/2, T = 4: (2/2) * sqrt(4) = 2
+    assert orc.muongs_ct_lower_bound(0.0, 4, 0.5, 4) == pytest.approx(2.0, rel=1e-15)
+    # r0 = 3, p = 16, eta = 1/4, T = 7: p eta^2 T = 7, sqrt(16) - 3 = 1, 2/(16/4) = 1/2
+    assert orc.muongs_ct_lower_bound(3.0, 16, 0.25, 7) == pytest.approx(0.5, rel=1e-15)
+    # r0 = 2, p = 3, eta = 1, T = 2: 2 p eta^2 T = 12, sqrt(16) = 4, eta T / 4 = 1/2
+    assert orc.muongs_late_lower_bound(2.0, 3, 1.0, 2) == pytest.approx(0.5, rel=1e-15)
+    # r0 = 0, p = 8, eta = 1/2, T = 1: 2 p eta^2 T = 4 -> 1/2 / 2 = 1/4
+    assert orc.muongs_late_lower_bound(0.0, 8, 0.5, 1) == pytest.approx(0.25, rel=1e-15)
+    assert orc.muonw_radius(1.0, 16, 2.0) == pytest.approx(2.0, rel=1e-15)   # sqrt(16)/2
+    assert orc.muonw_radius(5.0, 16, 2.0) == pytest.approx(5.0, rel=1e-15)   # r0 wins
+    assert orc.muonw_radius(0.5, 9, 0.5) == pytest.approx(6.0, rel=1e-15)    # sqrt(9)/0.5
+
+
+def test_muongs_bounds_are_tight_for_exact_polar_updates():
+    """Sandwich of Theorem 4.1 and Proposition 4.2 on a MuonGS run with the exact polar
+    factor (scale 1, wd 0, momentum 0 so that each update is independent of W_t). The
+    projection makes O~ orthogonal to W_t, so the norm recursion r_{t+1}^2 = r_t^2 +
+    eta^2 ||O~_t||^2 is exact and ||O~_t||^2 stays within a hair of p (independent random
+    gradients are almost orthogonal to W). With p_lo / p_hi the
+    smallest / largest ||O~_t||^2 of the run, for the decreasing 1/sqrt(.) sum:
+        bound_41(p_hi) <= C_T <= eta / r0 + bound_41(p_lo)
+    and the window C_2T - C_T lies between bound_42(p_hi) and 1.25 bound_42(p_lo)
+    (the exact sum over the window is 2 (sqrt 2 - 1) / (1/sqrt 2) = 1.17 times the
+    bound for large T). A loosened or mis-scaled bound (a factor 2, a dropped square
+    root, a missing p) falls outside one side."""
+    rng = np.random.default_rng(13)
+    rows, cols, eta, T = 64, 128, 0.02, 200
+    p = min(rows, cols)
+    W0 = rng.standard_normal((rows, cols)) * 0.02
+    grads = [rng.standard_normal((rows, cols)) * 1e-3 for _ in range(2 * T)]
+    hp = orc.HParams(lr=eta, momentum=0.0, mode="muongs", scale="none", exact_polar=True)
+    res = orc.muon_run(W0, grads, hp)
+    norms = [r.w_norm for r in res]
+    o2 = [r.o_norm ** 2 for r in res]
+    p_lo, p_hi = min(o2), max(o2)
+    assert p_hi <= p * (1 + 1e-12) and p_lo >= 0.99 * p
+    r0 = norms[0]
+    CT = orc.accumulated_lr([eta] * T, norms[:T])
+    C2T = orc.accumulated_lr([eta] * (2 * T), norms)
+    lo = orc.muongs_ct_lower_bound(r0, p_hi, eta, T)
+    hi = eta / r0 + orc.muongs_ct_lower_bound(r0, p_lo, eta, T)
+    assert lo <= CT <= hi
+    assert hi - lo <= 0.02 * CT        # the sandwich is narrow: the bound is tight here
+    assert orc.muongs_late_lower_bound(r0, p_hi, eta, T) <= C2T - CT
+    assert C2T - CT <= 1.25 * orc.muongs_late_lower_bound(r0, p_lo, eta, T)
+
+
+def test_muonw_radius_is_reached_by_an_aligned_update():
+    """Tightness of R_lambda = max(r0, sqrt(p)/lambda): with W_t = a_t Q for a fixed
+    semi-orthogonal Q (||Q||_F^2 = p) and the constant gradient -Q, the exact polar
+    update is O = -Q, so a_{t+1} = (1 - eta lambda) a_t + eta converges to 1/lambda and
+    ||W_t|| = a_t sqrt(p) rises to sqrt(p)/lambda from below, never above it."""
+    rows, cols, eta, lam, T = 8, 16, 0.05, 2.0, 400
+    p = min(rows, cols)
+    Q = orc.polar_factor(np.random.default_rng(14).standard_normal((rows, cols)))
+    W0 = 0.1 * Q
+    hp = orc.HParams(lr=eta, weight_decay=lam, scale="none", exact_polar=True)
+    res = orc.muon_run(W0, [-Q] * T, hp)
+    R = orc.muonw_radius(np.linalg.norm(W0), p, lam)
+    assert R == pytest.approx(np.sqrt(p) / lam, rel=1e-15)
+    assert all(r.w_norm <= R * (1 + 1e-12) for r in res)
+    assert np.linalg.norm(res[-1].W) == pytest.approx(R, rel=1e-9)
+
+
 def test_equilibration_hand_worked():
     """Rows of O have equal RMS (sqrt 3 each) so the columns are balanced:
     c = (sqrt(1/2), sqrt 2, sqrt(13/2)), rho = sqrt 3, O_ij <- O_ij rho / c_j."""

@@ -20,6 +20,7 @@
 #include "muon.h"
 #include "muon_internal.h"
 #include "ns_tc.h"
+#include "validate.h"
 
 using namespace muon;
 

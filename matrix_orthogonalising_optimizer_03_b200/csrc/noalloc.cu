@@ -28,6 +28,7 @@
 #include "muon.h"
 #include "muon_internal.h"
 #include "ns_tc.h"
+#include "validate.h"
 
 namespace muon {
 namespace {

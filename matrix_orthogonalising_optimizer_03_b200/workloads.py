@@ -195,6 +195,33 @@ def device_inputs(w: Workload, device, seed: int = 0, exact=(), step: int = 0):
     return Ws, Gs
 
 
+def device_grads(w: Workload, device, seed: int = 0, exact=(), step: int = 0):
+    """G_step for every matrix of a shape set, drawn on `device` from the distributions
+    `device_inputs` uses, with a generator of their own keyed by (seed, step) (the
+    weights are not drawn again). Matrices whose index is in `exact` get the host
+    generator's `grad(w, spec, step)` values, so that the oracle can follow them."""
+    import torch
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(np.random.SeedSequence([BASE_SEED, w.wid, seed, step, KIND_G])
+                        .generate_state(1)[0]))
+    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    exact = set(exact)
+    Gs = []
+    for spec in w.matrices():
+        shape = (spec.rows, spec.cols)
+        if spec.index in exact:
+            Gs.append(torch.from_numpy(grad(w, spec, step)).to(device=device, dtype=gdt))
+            continue
+        z = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+        if w.grad_dist == "student_t3":
+            v = torch.randn((3,) + shape, generator=gen, device=device, dtype=torch.float32)
+            z = z / torch.sqrt((v * v).mean(0))
+        elif w.grad_dist == "rowscaled":
+            z = z * torch.exp(torch.randn((spec.rows, 1), generator=gen, device=device))
+        Gs.append((z * w.g_std).to(gdt))
+    return Gs
+
+
 def sample_indices(w: Workload, extra: int = 8, seed: int = 7) -> List[int]:
     """One matrix per shape class (its first) plus `extra` seeded picks: the matrices a
     full-size parity check compares with the oracle one by one."""

@@ -70,6 +70,7 @@ class HParams:
     scale_k: float = 0.2
     equilibrate: bool = False
     exact_polar: bool = False    # replace the NS iteration by the SVD polar factor
+    equil_axis: Optional[int] = None  # force the equilibration axis (tests of near-ties)
 
 
 @dataclasses.dataclass
@@ -83,6 +84,7 @@ class StepResult:
     o_norm: float          # ||O_tilde||_F
     update_rms: float      # ||O_tilde||_F / sqrt(rows*cols)
     equil_axis: int
+    imbalances: Tuple[float, float] = (float("nan"), float("nan"))  # (rows, cols) before a6
 
 
 # ---------------------------------------------------------------- step a1-a2
@@ -153,7 +155,15 @@ def _imbalance(v: np.ndarray) -> float:
     return float(v.std() / mean) if mean > 0 else 0.0
 
 
-def equilibrate(O: np.ndarray, eps: float = 1e-7) -> Tuple[np.ndarray, int]:
+def line_imbalances(O: np.ndarray) -> Tuple[float, float]:
+    """(imbalance of the row RMS vector, imbalance of the column RMS vector) of O, the
+    two numbers `equilibrate` compares; imbalance(v) = std(v) / mean(v)."""
+    return (_imbalance(np.sqrt(np.mean(O * O, axis=1))),
+            _imbalance(np.sqrt(np.mean(O * O, axis=0))))
+
+
+def equilibrate(O: np.ndarray, eps: float = 1e-7, axis: Optional[int] = None
+                ) -> Tuple[np.ndarray, int]:
     """Row-or-column RMS equilibration of the orthogonalised update.
 
     [P4] section 핵심 내용: NorMuon normalises per row; MeqMuon picks row or column
@@ -164,11 +174,16 @@ def equilibrate(O: np.ndarray, eps: float = 1e-7) -> Tuple[np.ndarray, int]:
     O_ij <- O_ij * rho / (r_i + eps) (columns likewise), which keeps ||O||_F.
     Closed form: a line-scaled sign matrix D_r Z (or Z D_c) picks rows (columns) and maps
     to RMS(O) * Z. PARITY UNPINNED beyond that closed form and the invariants.
+    `axis` (AXIS_ROWS or AXIS_COLS) overrides the choice; the tests use it to follow the
+    other valid result when the two imbalances are a floating-point tie.
     """
     r = np.sqrt(np.mean(O * O, axis=1))
     c = np.sqrt(np.mean(O * O, axis=0))
     rho = np.sqrt(np.mean(O * O))
-    if _imbalance(r) >= _imbalance(c):
+    if axis is None:
+        ir, ic = line_imbalances(O)
+        axis = AXIS_ROWS if ir >= ic else AXIS_COLS
+    if axis == AXIS_ROWS:
         return O * (rho / (r + eps))[:, None], AXIS_ROWS
     return O * (rho / (c + eps))[None, :], AXIS_COLS
 
@@ -245,13 +260,15 @@ def muon_step(W: np.ndarray, G: np.ndarray, M_prev: np.ndarray, hp: HParams) -> 
     rows, cols = W.shape
     M, U = momentum(M_prev, G, hp.momentum, hp.nesterov)
     axis = AXIS_NONE
+    imb = (float("nan"), float("nan"))
     if hp.mode == "twosided":
         O = two_sided_normalise(frobenius_normalise(U, hp.eps), hp.eps)
         axis = 3
     else:
         O = orthogonalise(U, hp)
         if hp.equilibrate:
-            O, axis = equilibrate(O, hp.eps)
+            imb = line_imbalances(O)
+            O, axis = equilibrate(O, hp.eps, hp.equil_axis)
     O = update_scale(rows, cols, hp.scale, hp.scale_k) * O
     w_norm = float(np.linalg.norm(W))
     w_dot_o = float(np.sum(W * O))
@@ -261,7 +278,7 @@ def muon_step(W: np.ndarray, G: np.ndarray, M_prev: np.ndarray, hp: HParams) -> 
     if hp.mode == "muonh":
         W_next = retract_to_radius(W_next, w_norm)
     return StepResult(W_next, M, O, O_tilde, w_norm, w_dot_o, o_norm,
-                      o_norm / np.sqrt(rows * cols), axis)
+                      o_norm / np.sqrt(rows * cols), axis, imb)
 
 
 def muon_run(W0: np.ndarray, grads: Sequence[np.ndarray], hp: HParams,

@@ -299,6 +299,14 @@ def test_equilibration_hand_worked():
     got_t, axis_t = orc.equilibrate(O.T, eps=0.0)
     assert axis_t == orc.AXIS_ROWS
     assert np.allclose(got_t, got.T, rtol=0, atol=1e-15)
+    # row RMS (sqrt 3, sqrt 3): imbalance 0; column RMS above: imbalance > 0
+    ir, ic = orc.line_imbalances(O)
+    assert ir == 0.0 and ic > 0.3
+    # forcing the other axis scales the rows to rho: here the identity (r_i = rho)
+    forced, ax = orc.equilibrate(O, eps=0.0, axis=orc.AXIS_ROWS)
+    assert ax == orc.AXIS_ROWS and np.allclose(forced, O, rtol=0, atol=1e-15)
+    same, ax = orc.equilibrate(O, eps=0.0, axis=orc.AXIS_COLS)
+    assert ax == orc.AXIS_COLS and np.array_equal(same, got)
 
 
 @pytest.mark.parametrize("rows,cols", [(16, 16), (8, 24), (24, 8)])

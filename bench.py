@@ -2,17 +2,24 @@
 """Throughput of the Muon / MuonGS optimizer step on B200.
 
 One step = one pass of the whole step (momentum, normalisation, 5 Newton-Schulz
-iterations, scale, projection / decay, update) over every matrix of a shape set,
-with weights, momenta and gradients resident in HBM. Prints one JSON line.
+iterations, [equilibration], scale, projection / decay, update) over every matrix of
+a shape set, with weights, momenta and gradients resident in HBM. Prints one JSON
+line. The default shape set is the largest one that fits a GPU, the 1.5B dense set;
+the line also carries `per_set`, the same measurement for the other shape sets, and
+`sharded`, the ZeRO-1 sharded step over a one-rank NCCL group.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt160m]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dense_1p5b]
   python bench.py --impl reference ...   # the float64 CPU oracle on host cores
   python bench.py --impl torch ...       # the same step in eager PyTorch on the GPU
                                          # (cuBLAS bf16 batched matmuls), for comparison
 
-Multi-GPU (torchrun, one process per GPU): the matrices of a shape set are
-independent, so each rank steps its own copy of the shape set with no collective
-on the data path (weak scaling); `value` counts the shape-set steps of all ranks.
+Multi-GPU (torchrun, one process per GPU), `--dist sharded` (default): the ZeRO-1
+step of distributed.ShardedMuon over NCCL. Every rank holds its local gradients of
+every matrix; one reduce-scatter brings each matrix's averaged gradient to its owner,
+the owner runs the libmuon step on the matrices it owns, one all-gather shares the
+updated weights. One job step is one step of the whole shape set (strong scaling).
+`--dist replica`: every rank steps its own copy of the shape set with no collective
+on the data path (weak scaling). At N = 1 the headline is the plain plan step.
 """
 from __future__ import annotations
 
@@ -39,7 +46,12 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference", "torch"])
-    ap.add_argument("--workload", default="gpt160m")
+    ap.add_argument("--workload", default="dense_1p5b")
+    ap.add_argument("--dist", default="sharded", choices=["sharded", "replica"],
+                    help="multi-GPU mode: ZeRO-1 sharded step over NCCL, or independent replicas")
+    ap.add_argument("--no-per-set", action="store_true", help="skip the other shape sets")
+    ap.add_argument("--no-sharded", action="store_true",
+                    help="skip the one-rank NCCL sharded measurement at N = 1")
     ap.add_argument("--run", type=int, default=0,
                     help="which hyper-parameter setting of the workload (e.g. gpt400m: 0 MuonGS, 1 Muon+wd)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -309,10 +321,252 @@ def rank_max(x: float, world: int, device="cpu") -> float:
     return float(t.item())
 
 
-def throughput(steps: int, world: int, ms_max: float) -> float:
-    """Whole-job shape-set steps per second: every rank steps its own copy of the
-    shape set `steps` times (weak scaling), timed by the slowest rank."""
-    return steps * world / (ms_max / 1e3)
+def throughput(steps: int, world: int, ms_max: float, scaling: str = "weak") -> float:
+    """Whole-job shape-set steps per second, timed by the slowest rank. Weak scaling:
+    every rank steps its own copy of the shape set `steps` times. Strong scaling: the
+    ranks share one shape set, so a job step is one shape-set step."""
+    copies = world if scaling == "weak" else 1
+    return steps * copies / (ms_max / 1e3)
+
+
+# ------------------------------------------------------------------ per-kernel summaries
+ELEMENTWISE = ("ingest", "post_reduce", "post_apply")
+
+
+def elementwise_rates(prof, peaks):
+    """Achieved algorithmic GB/s of the memory-bound kernels and their fraction of the
+    measured HBM copy bandwidth."""
+    out = {}
+    for k in ELEMENTWISE:
+        v = prof.get(k)
+        if not v or not v["launches"] or v["total_ms"] <= 0:
+            continue
+        gbs = v["bytes"] / (v["total_ms"] / 1e3) / 1e9
+        out[k] = {"gb_s": gbs, "frac": gbs / peaks["hbm_gbs"],
+                  "bytes_per_launch": v["bytes"] / v["launches"],
+                  "ms_per_launch": v["total_ms"] / v["launches"]}
+    return out
+
+
+def ns_rates(prof, w, steps: int, ms_total: float, peaks):
+    """Newton-Schulz throughput in algorithmic flops (symmetric Gram and polynomial
+    counted once), over the whole step time and over the summed time of the
+    Newton-Schulz launches, each as a fraction of the burst and sustained bf16 peaks."""
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+    flops = wl.workload_ns_flops(w) * steps
+    ns_ms = sum(v["total_ms"] for k, v in prof.items() if k.startswith("ns_"))
+    step_tf = flops / (ms_total / 1e3) / 1e12
+    phase_tf = flops / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
+
+    def fr(x):
+        if x is None or w.ns_fp32:
+            return None
+        return {"burst": x / peaks["bf16_tflops"], "sustained": x / peaks["bf16_tflops_sustained"]}
+    return {"ns_tflops_step": step_tf, "ns_frac_step": fr(step_tf),
+            "ns_tflops_phases": phase_tf, "ns_frac_phases": fr(phase_tf),
+            "ns_ms_per_step": ns_ms / steps}
+
+
+# ------------------------------------------------------------------ one shape set on one GPU
+def set_inputs(w, dev, seed: int):
+    """Resident inputs of a shape set: W (fp32), M (fp32, zero) and one flat gradient
+    buffer with a view per matrix, drawn on the device (seeded)."""
+    import torch
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+    specs = w.matrices()
+    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    numel = sum(s.rows * s.cols for s in specs)
+    Ws, G_src = wl.device_inputs(w, dev, seed=seed)
+    g_flat = torch.empty(numel, dtype=gdt, device=dev)
+    Ms, Gs = [], []
+    off = 0
+    for s, g in zip(specs, G_src):
+        Ms.append(torch.zeros(s.rows, s.cols, dtype=torch.float32, device=dev))
+        gv = g_flat[off:off + s.rows * s.cols].view(s.rows, s.cols)
+        gv.copy_(g)
+        Gs.append(gv)
+        off += s.rows * s.cols
+    del G_src
+    return Ws, Gs, Ms, g_flat, numel, gdt
+
+
+def time_steps(step, steps: int, world: int, dev, stream, after_start=None):
+    """CUDA-event time (ms, max over ranks) of `steps` calls of step(), bracketed by a
+    barrier and a device synchronisation on both sides. after_start() runs right after
+    the start event is recorded (e.g. to order another stream behind it)."""
+    import torch
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    if after_start is not None:
+        after_start()
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    barrier()
+    return rank_max(e0.elapsed_time(e1), world, dev)
+
+
+def measure_plan(B, w, run, args, dev, world: int, peaks, peak_src, seed: int, full: bool):
+    """The plain plan step of one shape set: warm-up, K timed steps, K profiled steps
+    (per-kernel CUDA events), and with `full` the end-to-end feed. Returns a summary
+    dict and the live objects the caller may reuse (weights, momenta, plan)."""
+    import torch
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+    Ws, Gs, Ms, g_flat, numel, gdt = set_inputs(w, dev, seed)
+    gsz = 2 if w.grad_dtype == "bf16" else 4
+    hp = B.hparams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
+                   equilibrate=run.equilibrate, ns_fp32=w.ns_fp32)
+    plan = B.Plan(Ws, Gs, Ms, hp)
+    stats = B.new_stats(len(Ws), dev)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    local = dev.index if dev.index is not None else 0
+    sampler = ClockSampler(gpu_id_for(torch, local))
+    for _ in range(args.warmup):
+        plan.step(stats=stats)
+    torch.cuda.synchronize()
+    if plan.query_device_status() != 0:
+        raise RuntimeError(f"device-side error during warm-up ({w.name})")
+    ms = time_steps(lambda: plan.step(stats=stats), args.steps, world, dev, stream)
+    clocks = sampler.stop()
+    # profiled pass over the same K steps: per-kernel device times on the launching stream
+    B.load().muon_plan_profile_enable(plan._plan, 1)
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        plan.step(stats=stats)
+    prof = plan_profile(B, plan)
+    B.load().muon_plan_profile_enable(plan._plan, 0)
+    launches = sum(p["launches"] for p in prof.values())
+    out = {
+        "value": throughput(args.steps, world, ms, "weak"), "unit": "steps/s",
+        "ms_per_step": ms / args.steps, "matrices": w.n_matrices, "params": w.n_params,
+        "mode": run.mode, "weight_decay": run.weight_decay, "equilibrate": run.equilibrate,
+        "ns_path": "fp32 CUDA cores" if w.ns_fp32 else "bf16 tcgen05",
+        **ns_rates(prof, w, args.steps, ms, peaks),
+        "roofline": roofline(prof, w, peaks, peak_src, w.name, ms),
+        "elementwise": elementwise_rates(prof, peaks),
+        "kernels": {k: {"launches_per_step": v["launches"] / args.steps,
+                        "ms_per_step": v["total_ms"] / args.steps} for k, v in prof.items()
+                    if v["launches"]},
+        "gpu_launches": int(round(launches)),
+        "clocks": clocks,
+        "l2": "inputs larger than L2 (W+M+G = %.0f MB vs 126 MB)" % (numel * (8 + gsz) / 1e6),
+    }
+    if full:
+        # end to end through the public API (binding.StreamedSteps): every step copies
+        # its gradients from pinned host memory and reads the per-matrix statistics
+        # back; the copy of step t+1 overlaps step t on a second stream
+        g_host = torch.empty(numel, dtype=gdt, pin_memory=True)
+        g_host.copy_(g_flat)
+        feed = B.StreamedSteps(Ws, Ms, hp, grad_dtype=gdt)
+        for _ in range(2):
+            feed.step(g_host)
+
+        def fed_step():
+            feed.step(g_host)
+        # every copy starts inside the timed region: the copy stream waits for the start
+        ms_e2e = time_steps(fed_step, args.steps, world, dev, stream,
+                            after_start=lambda: feed.copy_stream.wait_stream(stream))
+        torch.cuda.synchronize()
+        feed.close()
+        del feed, g_host
+        out["e2e"] = {"value": throughput(args.steps, world, ms_e2e, "weak"), "unit": "steps/s",
+                      "h2d_bytes_per_step": numel * gsz, "d2h_bytes_per_step": stats.numel() * 4,
+                      "overlap": "H2D of step t+1 on a copy stream during step t (two buffers)"}
+    if plan.query_device_status() != 0:
+        raise RuntimeError(f"device-side error in the timed region ({w.name})")
+    plan.close()
+    del plan, Gs, g_flat, stats
+    return out, Ws, Ms
+
+
+def measure_sharded(B, w, run, args, dev, world: int, rank: int, peaks, peak_src, seed: int,
+                    e2e: bool):
+    """The ZeRO-1 sharded step (distributed.ShardedMuon) over the current NCCL process
+    group: reduce-scatter of the gradients to their owners, the owners' libmuon plan
+    step, all-gather of the updated weights. Every rank holds its own local gradients
+    of every matrix. One job step is one shape-set step (strong scaling)."""
+    import torch
+    from matrix_orthogonalising_optimizer_03_b200 import distributed as D
+    from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
+    specs = w.matrices()
+    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    gsz = 2 if w.grad_dtype == "bf16" else 4
+    Ws, Gs = wl.device_inputs(w, dev, seed=seed)
+    opt = D.ShardedMuon([(s.rows, s.cols) for s in specs], dev, init=Ws, grad_dtype=gdt,
+                        lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay,
+                        mode=run.mode, equilibrate=run.equilibrate, ns_fp32=w.ns_fp32)
+    for gv, g in zip(opt.grads, Gs):
+        gv.copy_(g)
+    del Ws, Gs
+    n_mine = len(opt.mine)
+    stats = B.new_stats(max(n_mine, 1), dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        opt.step(stats=stats if n_mine else None)
+    torch.cuda.synchronize()
+    local = dev.index if dev.index is not None else 0
+    sampler = ClockSampler(gpu_id_for(torch, local))
+    ms = time_steps(lambda: opt.step(stats=stats if n_mine else None), args.steps, world, dev,
+                    stream)
+    clocks = sampler.stop()
+    prof = {}
+    if opt.plan is not None:
+        B.load().muon_plan_profile_enable(opt.plan._plan, 1)
+        torch.cuda.synchronize()
+    for _ in range(args.steps):   # every rank takes part in the collectives
+        opt.step(stats=stats if n_mine else None)
+    if opt.plan is not None:
+        prof = plan_profile(B, opt.plan)
+        B.load().muon_plan_profile_enable(opt.plan._plan, 0)
+    launches = rank_max(float(sum(p["launches"] for p in prof.values())), world, dev)
+    out = {"value": throughput(args.steps, world, ms, "strong"), "unit": "steps/s",
+           "ms_per_step": ms / args.steps, "world": world, "backend": opt.backend,
+           "scaling": "strong", "owned_matrices": n_mine,
+           "collectives": "reduce_scatter_tensor (avg, bf16 grads) + all_gather_into_tensor "
+                          "(fp32 W), in place",
+           "kernels": {k: {"launches_per_step": v["launches"] / args.steps,
+                           "ms_per_step": v["total_ms"] / args.steps} for k, v in prof.items()
+                       if v["launches"]},
+           "gpu_launches_max_rank": int(round(launches)),
+           "clocks": clocks}
+    if prof:
+        out["roofline"] = roofline(prof, w, peaks, peak_src, w.name, ms)
+    if e2e:
+        # end to end: each step copies this rank's local gradients from pinned host
+        # memory (on the compute stream, not overlapped) and reads the statistics back
+        numel = opt.flat_g.numel()
+        g_host = torch.empty(numel, dtype=gdt, pin_memory=True)
+        g_host.copy_(opt.flat_g)
+        st_host = torch.empty_like(stats, device="cpu").pin_memory()
+
+        def fed_step():
+            opt.flat_g.copy_(g_host, non_blocking=True)
+            opt.step(stats=stats if n_mine else None)
+            st_host.copy_(stats, non_blocking=True)
+        ms_e2e = time_steps(fed_step, args.steps, world, dev, stream)
+        out["e2e"] = {"value": throughput(args.steps, world, ms_e2e, "strong"), "unit": "steps/s",
+                      "h2d_bytes_per_step": numel * gsz, "d2h_bytes_per_step": stats.numel() * 4,
+                      "overlap": "none (copy, step and read-back in order on one stream)"}
+        del g_host, st_host
+    if opt.plan is not None:
+        if opt.plan.query_device_status() != 0:
+            raise RuntimeError("device-side error in the sharded step")
+        opt.plan.close()
+    del opt
+    torch.cuda.synchronize()
+    return out
+
+
+PER_SET = [("gpt160m", 0), ("gpt400m", 0), ("gpt400m", 1), ("moe_1b", 0), ("single_128x256", 0),
+           ("single_128x256", 1)]
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -326,7 +580,6 @@ def main():
     if args.impl == "torch":
         return run_torch(args, rank, world, local)
 
-    import numpy as np
     import torch
     import torch.distributed as dist
     from datetime import timedelta
@@ -341,124 +594,85 @@ def main():
     B.load()
     w = wl.WORKLOADS[args.workload]
     run = w.runs[args.run]
-    specs = w.matrices()
-    gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
+    peaks, peak_src = load_peaks()
+    sharded_job = world > 1 and args.dist == "sharded"
     gsz = 2 if w.grad_dtype == "bf16" else 4
 
-    # resident inputs: W (fp32), M (fp32, zero), G (one flat buffer, views per matrix),
-    # drawn on the device from the shape set's distributions (seeded)
-    numel = sum(s.rows * s.cols for s in specs)
-    Ws, G_src = wl.device_inputs(w, dev, seed=rank)
-    g_flat = torch.empty(numel, dtype=gdt, device=dev)
-    Ms, Gs = [], []
-    off = 0
-    for s, g in zip(specs, G_src):
-        Ms.append(torch.zeros(s.rows, s.cols, dtype=torch.float32, device=dev))
-        gv = g_flat[off:off + s.rows * s.cols].view(s.rows, s.cols)
-        gv.copy_(g)
-        Gs.append(gv)
-        off += s.rows * s.cols
-    del G_src
-    g_host = torch.empty(numel, dtype=gdt, pin_memory=True)
-    g_host.copy_(g_flat)
-    hp = B.hparams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
-                   equilibrate=run.equilibrate, ns_fp32=w.ns_fp32)
-    plan = B.Plan(Ws, Gs, Ms, hp)
-    stats = B.new_stats(len(specs), dev)
-    stream = torch.cuda.current_stream()
-    torch.cuda.synchronize()
+    if sharded_job:
+        res = measure_sharded(B, w, run, args, dev, world, rank, peaks, peak_src, 0, e2e=True)
+        line_core = {"value": res["value"], "ms_per_step": res["ms_per_step"],
+                     "scaling": "strong", "roofline": res.get("roofline"),
+                     "kernels": res["kernels"], "gpu_launches": res["gpu_launches_max_rank"],
+                     "e2e": res["e2e"], "clocks": res["clocks"]}
+        parallelism = f"zero1-sharded x{world} (nccl)"
+        extra = {"sharded": {k: v for k, v in res.items() if k not in ("e2e",)}}
+        cpu = None
+    else:
+        res, _, _ = measure_plan(B, w, run, args, dev, world, peaks, peak_src, rank, full=True)
+        line_core = {"value": res["value"], "ms_per_step": res["ms_per_step"],
+                     "scaling": "weak" if world > 1 else "strong", "roofline": res["roofline"],
+                     "kernels": res["kernels"], "gpu_launches": res["gpu_launches"],
+                     "e2e": res["e2e"], "clocks": res["clocks"]}
+        parallelism = f"replica x{world}" if world > 1 else "single GPU"
+        extra = {k: res[k] for k in ("ns_tflops_step", "ns_frac_step", "ns_tflops_phases",
+                                     "ns_frac_phases", "ns_ms_per_step", "elementwise")}
+        cpu = None
+        if world == 1 and rank == 0 and not args.no_cpu_baseline:
+            est, n, rounds = oracle_sample(w, run, args.cpu_seconds)
+            cpu = {"value": 1.0 / est, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                   "sample": f"float64 oracle on {n} matrices ({rounds} per shape class) of the "
+                             f"{w.name} shape set, extrapolated to one full step by class counts"}
+        torch.cuda.empty_cache()
+        if world == 1 and not args.no_sharded:
+            # the sharded step at world 1: a one-rank NCCL group, in-place collectives
+            dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                                    device_id=dev)
+            try:
+                sh = measure_sharded(B, w, run, args, dev, 1, 0, peaks, peak_src, 0, e2e=False)
+            finally:
+                dist.destroy_process_group()
+            extra["sharded"] = {k: sh[k] for k in ("value", "unit", "ms_per_step", "world",
+                                                   "backend", "scaling", "collectives",
+                                                   "gpu_launches_max_rank")}
+            torch.cuda.empty_cache()
+        if world == 1 and not args.no_per_set:
+            per = {}
+            for name, ridx in PER_SET:
+                if name == w.name and ridx == args.run:
+                    continue
+                ws = wl.WORKLOADS[name]
+                r, _, _ = measure_plan(B, ws, ws.runs[ridx], args, dev, 1, peaks, peak_src, 0,
+                                       full=False)
+                r.pop("kernels", None)
+                per[f"{name}/{ws.runs[ridx].mode}" + ("+wd" if ws.runs[ridx].weight_decay else "")] = r
+                torch.cuda.empty_cache()
+            extra["per_set"] = per
 
-    sampler = ClockSampler(gpu_id_for(torch, local))
-    for _ in range(args.warmup):
-        plan.step(stats=stats)
-    torch.cuda.synchronize()
-    if plan.query_device_status() != 0:
-        raise RuntimeError("device-side error during warm-up")
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(x: float) -> float:
-        return rank_max(x, world, dev)
-
-    # 1) device-timed region: K steps, inputs resident (W+M+G far larger than L2)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        plan.step(stats=stats)
-    e1.record(stream)
-    barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1))
-    clocks = sampler.stop()
-
-    # 2) profiled pass (same K steps): per-kernel device times on the launching stream
-    B.load().muon_plan_profile_enable(plan._plan, 1)
-    barrier()
-    for _ in range(args.steps):
-        plan.step(stats=stats)
-    prof = plan_profile(B, plan)
-    B.load().muon_plan_profile_enable(plan._plan, 0)
-    launches_per_step = sum(p["launches"] for p in prof.values()) / args.steps
-
-    # 3) end to end through the public API (binding.StreamedSteps): every step copies
-    #    its gradients from pinned host memory and reads the per-matrix statistics
-    #    back; the copy of step t+1 overlaps step t on a second stream
-    feed = B.StreamedSteps(Ws, Ms, hp, grad_dtype=gdt)
-    for _ in range(2):
-        feed.step(g_host)
-    barrier()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    feed.copy_stream.wait_stream(stream)   # every copy starts inside the timed region
-    for _ in range(args.steps):
-        feed.step(g_host)
-    stream.wait_stream(feed.copy_stream)
-    f1.record(stream)
-    barrier()
-    ms_e2e = max_over_ranks(f0.elapsed_time(f1))
-    feed.close()
-    if plan.query_device_status() != 0:
-        raise RuntimeError("device-side error in the timed region")
-
-    peaks, peak_src = load_peaks()
-    roof = roofline(prof, w, peaks, peak_src, args.workload, ms)
-    cpu = None
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        est, n, rounds = oracle_sample(w, run, args.cpu_seconds)
-        cpu = {"value": 1.0 / est, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"float64 oracle on {n} matrices ({rounds} per shape class) of the "
-                         f"{w.name} shape set, extrapolated to one full step by class counts"}
     if rank == 0:
         line = {
-            "metric": "muon_steps_per_s", "value": throughput(args.steps, world, ms), "unit": "steps/s",
+            "metric": "muon_steps_per_s", "value": line_core["value"], "unit": "steps/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32" if w.ns_fp32 else "bf16", "data": "synthetic",
+            "ms_per_step": line_core["ms_per_step"], "higher_is_better": True,
+            "scaling": line_core["scaling"], "vs_baseline": None,
+            "dtype": "f32" if w.ns_fp32 else "bf16", "data": "synthetic",
             "config": {"workload": w.name, "matrices": w.n_matrices, "params": w.n_params,
                        "mode": run.mode, "weight_decay": run.weight_decay,
                        "equilibrate": run.equilibrate, "ns_steps": 5, "grad_dtype": w.grad_dtype,
                        "ns_path": "fp32 CUDA cores" if w.ns_fp32 else "bf16 tcgen05",
                        "ns_tflops_per_step": wl.workload_ns_flops(w) / 1e12,
                        "l2": "inputs larger than L2 (W+M+G = %.0f MB vs 126 MB)" % (
-                           numel * (8 + gsz) / 1e6),
-                       "parallelism": f"replica x{world}"},
-            "ns_tflops": wl.workload_ns_flops(w) * args.steps / (ms / 1e3) / 1e12,
-            "roofline": roof,
-            "kernels": {k: {"launches_per_step": v["launches"] / args.steps,
-                            "ms_per_step": v["total_ms"] / args.steps} for k, v in prof.items()
-                        if v["launches"]},
-            "gpu_launches": int(round(launches_per_step * args.steps)),
-            "e2e": {"value": throughput(args.steps, world, ms_e2e), "unit": "steps/s",
-                    "h2d_bytes_per_step": numel * gsz, "d2h_bytes_per_step": stats.numel() * 4,
-                    "overlap": "H2D of step t+1 on a copy stream during step t (two buffers)"},
-            "clocks": clocks,
+                           w.n_params * (8 + gsz) / 1e6),
+                       "parallelism": parallelism},
+            "ns_tflops": extra.get("ns_tflops_step"),
+            "roofline": line_core["roofline"],
+            "kernels": line_core["kernels"],
+            "gpu_launches": line_core["gpu_launches"],
+            "e2e": line_core["e2e"],
+            "clocks": line_core["clocks"],
             "cpu_baseline": cpu,
+            **extra,
         }
         print(json.dumps(line), flush=True)
-    plan.close()
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

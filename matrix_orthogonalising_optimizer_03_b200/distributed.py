@@ -17,9 +17,13 @@ one reduce-scatter and one all-gather move everything:
     owned  [rank r matrices | pad]  --local Muon step (libmuon, in place on W)-->
     W      [rank 0 matrices | pad][rank 1 ...]   <--all-gather of each owner's segment
 
-On NCCL the collectives are reduce_scatter_tensor / all_gather_into_tensor; on
-gloo (CPU tests) the same data movement is done with all_reduce + slicing and
-all_gather. The per-matrix parameter and gradient tensors handed out are views
+On NCCL the collectives are reduce_scatter_tensor / all_gather_into_tensor, both in
+place (this rank's segment of the flat buffer is the reduce-scatter's output and the
+all-gather's input, NCCL's in-place forms), so a step allocates and copies nothing
+beyond the collectives themselves. They run whenever a process group exists, a
+single-rank NCCL group included. On gloo (CPU tests) the same data movement is done
+with all_reduce + slicing and all_gather. Without a process group the step is the
+local step alone. The per-matrix parameter and gradient tensors handed out are views
 into the flat buffers, so a training loop writes gradients in place and reads the
 updated weights without copies.
 """
@@ -60,9 +64,10 @@ class ShardedMuon:
         import torch
         import torch.distributed as dist
         self.torch, self.dist = torch, dist
-        self.world = dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
-        self.rank = dist.get_rank() if self.world > 1 else 0
-        self.backend = dist.get_backend() if self.world > 1 else None
+        self.grouped = dist.is_available() and dist.is_initialized()
+        self.world = dist.get_world_size() if self.grouped else 1
+        self.rank = dist.get_rank() if self.grouped else 0
+        self.backend = dist.get_backend() if self.grouped else None
         self.device = torch.device(device)
         self.shapes = [tuple(s) for s in shapes]
         self.owner = lpt_partition([wl.ns_flops(r, c) for r, c in self.shapes], self.world)
@@ -80,7 +85,10 @@ class ShardedMuon:
         n = self.seg * self.world
         self.flat_w = torch.zeros(n, dtype=torch.float32, device=self.device)
         self.flat_g = torch.zeros(n, dtype=gdt, device=self.device)
-        self.my_g = torch.zeros(self.seg, dtype=gdt, device=self.device)
+        # this rank's segment: the in-place reduce-scatter leaves the averaged gradients
+        # of the matrices it owns here
+        self.my_g = self.flat_g[self.rank * self.seg:(self.rank + 1) * self.seg]
+        self.my_w = self.flat_w[self.rank * self.seg:(self.rank + 1) * self.seg]
         self.params, self.grads = [], []
         for i, (r, c) in enumerate(self.shapes):
             base = self.owner[i] * self.seg + self.offsets[i]
@@ -105,9 +113,8 @@ class ShardedMuon:
     # -- collectives ------------------------------------------------------------
     def _reduce_scatter_grads(self):
         dist = self.dist
-        if self.world == 1:
-            self.my_g.copy_(self.flat_g[:self.seg])
-            return
+        if not self.grouped:
+            return                          # one process: my_g is the whole buffer
         if self.backend == "nccl":
             dist.reduce_scatter_tensor(self.my_g, self.flat_g, op=dist.ReduceOp.AVG)
             return
@@ -117,14 +124,13 @@ class ShardedMuon:
 
     def _all_gather_weights(self):
         dist = self.dist
-        if self.world == 1:
+        if not self.grouped:
             return
-        mine = self.flat_w[self.rank * self.seg:(self.rank + 1) * self.seg]
         if self.backend == "nccl":
-            dist.all_gather_into_tensor(self.flat_w, mine.clone())
+            dist.all_gather_into_tensor(self.flat_w, self.my_w)
             return
         parts = list(self.flat_w.split(self.seg))
-        dist.all_gather(parts, mine.clone())
+        dist.all_gather(parts, self.my_w.clone())
 
     # -- one optimizer step -----------------------------------------------------
     def step(self, stats=None):

@@ -110,3 +110,42 @@ def test_single_rank_sharded_step_runs_libmuon(lib):
     for a, b in zip(opt.params, Ws):
         assert torch.allclose(a, b, rtol=0, atol=1e-6)
     plan.close()
+
+
+@pytest.mark.gpu
+def test_single_rank_nccl_sharded_steps_match_oracle(lib):
+    """The NCCL branch (in-place reduce_scatter_tensor and all_gather_into_tensor) on a
+    one-rank NCCL process group, with the libmuon plan as the owner's step: three MuonGS
+    steps, each weight against the float64 oracle at the bf16 path's tolerance."""
+    import torch
+    import torch.distributed as dist
+    from oracle import muon_oracle as orc
+    from tests import gpu_helpers as H
+    shapes = [(256, 512), (768, 256), (100, 70), (512, 512)]
+    W0 = [wl.normal(r, c, 40 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[wl.normal(r, c, 50 + 10 * t + i, 1e-3, bf16=True) for i, (r, c) in enumerate(shapes)]
+             for t in range(3)]
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        opt = D.ShardedMuon(shapes, "cuda", init=[torch.from_numpy(w) for w in W0], mode="muongs")
+        assert opt.grouped and opt.backend == "nccl"
+        got = []
+        for t in range(3):
+            for g_view, g in zip(opt.grads, grads[t]):
+                g_view.copy_(torch.from_numpy(g))
+            opt.step()
+            torch.cuda.synchronize()
+            got.append([p.double().cpu().numpy() for p in opt.params])
+        assert opt.plan.query_device_status() == 0
+        opt.plan.close()
+    finally:
+        dist.destroy_process_group()
+    hp = orc.HParams(mode="muongs")
+    for i in range(len(shapes)):
+        res = orc.muon_run(W0[i], [g[i] for g in grads], hp)
+        W_prev_g = W_prev_o = W0[i].astype(np.float64)
+        for t, r in enumerate(res):
+            assert H.rel(got[t][i], r.W) <= H.TOL_BF16
+            assert H.rel(W_prev_g - got[t][i], W_prev_o - r.W) <= H.TOL_BF16, (i, t)
+            W_prev_g, W_prev_o = got[t][i], r.W

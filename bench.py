@@ -460,6 +460,20 @@ def measure_plan(B, w, run, args, dev, world: int, peaks, peak_src, seed: int, f
         "l2": "inputs larger than L2 (W+M+G = %.0f MB vs 126 MB)" % (numel * (8 + gsz) / 1e6),
     }
     if full:
+        # a learning-rate schedule: new hyper-parameters before every step (the plan
+        # updates its captured graph in place)
+        lrs = [w.lr * (0.5 + 0.5 * ((t * 7) % 10) / 10.0) for t in range(args.steps)]
+        it = iter(lrs)
+
+        def sched_step():
+            plan.set_hparams(B.hparams(lr=next(it), momentum=w.momentum,
+                                       weight_decay=run.weight_decay, mode=run.mode,
+                                       equilibrate=run.equilibrate, ns_fp32=w.ns_fp32))
+            plan.step(stats=stats)
+        ms_sched = time_steps(sched_step, args.steps, world, dev, stream)
+        out["lr_schedule"] = {"value": throughput(args.steps, world, ms_sched, "weak"),
+                              "unit": "steps/s", "ms_per_step": ms_sched / args.steps,
+                              "what": "muon_plan_set_hparams (new lr) before every step"}
         # end to end through the public API (binding.StreamedSteps): every step copies
         # its gradients from pinned host memory and reads the per-matrix statistics
         # back; the copy of step t+1 overlaps step t on a second stream
@@ -615,7 +629,8 @@ def main():
                      "e2e": res["e2e"], "clocks": res["clocks"]}
         parallelism = f"replica x{world}" if world > 1 else "single GPU"
         extra = {k: res[k] for k in ("ns_tflops_step", "ns_frac_step", "ns_tflops_phases",
-                                     "ns_frac_phases", "ns_ms_per_step", "elementwise")}
+                                     "ns_frac_phases", "ns_ms_per_step", "elementwise",
+                                     "lr_schedule")}
         cpu = None
         if world == 1 and rank == 0 and not args.no_cpu_baseline:
             est, n, rounds = oracle_sample(w, run, args.cpu_seconds)

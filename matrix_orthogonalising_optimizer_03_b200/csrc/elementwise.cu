@@ -12,12 +12,12 @@
 //
 // Work unit: a 128 x 256 super-tile of the matrix in its storage frame per
 // 256-thread block, walked as 4 x 4 sub-tiles of 32 x 64 (8 consecutive columns
-// per thread, 128-bit accesses when aligned; the plain reduction and post_apply
-// take two 32-row sub-tiles at a time). The super-tile of each block is found by
-// binary search over a per-matrix tile prefix. Per-matrix sums use one
-// atomic per block; the equilibration row / column sums are reduced inside the
-// block (shuffles for rows, a shared-memory transpose for columns) and use one
-// atomic per row and per column of the super-tile.
+// per thread, 128-bit accesses when aligned; the reductions and post_apply take two
+// 32-row sub-tiles at a time, all their loads issued before any arithmetic). The
+// super-tile of each block is found by binary search over a per-matrix tile prefix.
+// Per-matrix sums use one atomic per block; the equilibration row / column sums are
+// reduced inside the block (shuffles, and shared memory across warps for columns) and
+// use one atomic per row and per column of the super-tile.
 #include <cuda_runtime.h>
 
 #include "muon_internal.h"
@@ -109,40 +109,6 @@ __device__ __forceinline__ void block_sum(double (&v)[NV], double (*sh)[kThreads
       double x = lane < kThreads / 32 ? sh[i][lane] : 0.0;
       v[i] = warp_sum(x);
     }
-  }
-}
-
-// Loads, for this thread's 8 storage-frame elements, the Newton-Schulz result O.
-// Tall matrices hold O^T in the slab: the block stages a 64 x 32 slab tile in
-// shared memory and reads it transposed. Block-uniform control flow.
-__device__ __forceinline__ void load_o_tile(const ElemArgs& a, const DevMat& d, const DevSlab& s,
-                                            int r0, int c0, float (*tile)[kTR + 1],
-                                            float (&o)[8]) {
-  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
-  const int r = r0 + lr, c = c0 + lc;
-  if (!(d.flags & MAT_TRANSPOSED)) {
-    const int valid = (r < d.rows) ? min(8, d.cols - c) : 0;
-    if (valid > 0) load8_slab(s.xf, a.x_fp32, (int64_t)r * s.ldx + c, valid, o);
-    else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[e] = 0.f;
-    }
-  } else {
-    // slab rows = storage columns c0..c0+63, slab columns = storage rows r0..r0+31
-    const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
-    float v[8];
-    const int valid = (sr < d.cols) ? min(8, d.rows - sc) : 0;
-    if (valid > 0) load8_slab(s.xf, a.x_fp32, (int64_t)sr * s.ldx + sc, valid, v);
-    else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] = 0.f;
-    }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) tile[threadIdx.x >> 2][(threadIdx.x & 3) * 8 + e] = v[e];
-    __syncthreads();
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[e] = tile[lc + e][lr];
-    __syncthreads();  // the tile is reused by the next sub-tile
   }
 }
 
@@ -238,108 +204,6 @@ __device__ __forceinline__ float slab_scale(const ElemArgs& a, int k) {
   return static_cast<float>(1.0 / (sqrt(a.scal[k].u2) + (double)a.eps));
 }
 
-// ------------------------------------------------------------------ post_reduce (equilibration)
-// Equilibration and the two-sided mode: the three per-matrix sums plus the per-row and
-// per-column sums of O^2 and W*O.
-__global__ void __launch_bounds__(kThreads, 4) post_reduce_eq_kernel(const ElemArgs a) {
-  griddep_launch_dependents();
-  griddep_wait();
-  __shared__ float tile[kTC][kTR + 1];
-  __shared__ double red[3][kThreads / 32];
-  __shared__ float colred[2][kTR][kTC + 1];
-  const int b = blockIdx.x;
-  const int k = find_matrix(a, b);
-  const DevMat d = a.mats[k];
-  const DevSlab s = a.slabs[k];
-  const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
-  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
-  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
-  const bool vec = (d.flags & MAT_VEC_OK) != 0;
-  const float xs = slab_scale(a, k);
-  float ww = 0.f, wo = 0.f, oo = 0.f;
-  float row_o2[kSubR], row_wo[kSubR];  // this thread's share of its rows' sums
-#pragma unroll
-  for (int i = 0; i < kSubR; ++i) row_o2[i] = row_wo[i] = 0.f;
-
-  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
-    const int c0 = C0 + bj * kTC;
-    float col_o2[8], col_wo[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) col_o2[e] = col_wo[e] = 0.f;
-#pragma unroll
-    for (int bi = 0; bi < kSubR; ++bi) {
-      const int r0 = R0 + bi * kTR;
-      if (r0 >= d.rows) break;  // uniform over the block
-      const int r = r0 + lr, c = c0 + lc;
-      const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
-      float o[8];
-      load_o_tile(a, d, s, r0, c0, tile, o);
-      float w[8];
-      if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w);
-      else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w[e] = 0.f;
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float oe = e < valid ? o[e] * xs : 0.f;
-        ww = fmaf(w[e], w[e], ww);
-        wo = fmaf(w[e], oe, wo);
-        oo = fmaf(oe, oe, oo);
-        if (a.equilibrate) {
-          row_o2[bi] = fmaf(oe, oe, row_o2[bi]);
-          row_wo[bi] = fmaf(w[e], oe, row_wo[bi]);
-          col_o2[e] = fmaf(oe, oe, col_o2[e]);
-          col_wo[e] = fmaf(w[e], oe, col_wo[e]);
-        }
-      }
-    }
-    if (a.equilibrate) {
-      // column sums over the super-tile's rows: transpose through shared memory
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        colred[0][lr][lc + e] = col_o2[e];
-        colred[1][lr][lc + e] = col_wo[e];
-      }
-      __syncthreads();
-      if (threadIdx.x < 2 * kTC) {
-        const int which = threadIdx.x / kTC, cc = threadIdx.x % kTC;
-        float sum = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < kTR; ++i) sum += colred[which][i][cc];
-        if (c0 + cc < d.cols)
-          atomicAdd((which ? a.eq_wo : a.eq_o2) + s.eq_off + d.rows + c0 + cc, sum);
-      }
-      __syncthreads();
-    }
-  }
-  if (a.equilibrate) {
-    // row sums: the 8 threads of a row are consecutive lanes
-#pragma unroll
-    for (int bi = 0; bi < kSubR; ++bi) {
-      float ro = row_o2[bi], rw = row_wo[bi];
-#pragma unroll
-      for (int m = 4; m > 0; m >>= 1) {
-        ro += __shfl_xor_sync(0xffffffffu, ro, m);
-        rw += __shfl_xor_sync(0xffffffffu, rw, m);
-      }
-      const int r = R0 + bi * kTR + lr;
-      if ((threadIdx.x & 7) == 0 && r < d.rows) {
-        atomicAdd(a.eq_o2 + s.eq_off + r, ro);
-        atomicAdd(a.eq_wo + s.eq_off + r, rw);
-      }
-    }
-  }
-  double acc[3] = {ww, wo, oo};
-  block_sum<3>(acc, red);
-  if (threadIdx.x == 0) {
-    atomicAdd(&a.scal[k].w2, acc[0]);
-    atomicAdd(&a.scal[k].wo, acc[1]);
-    atomicAdd(&a.scal[k].o2, acc[2]);
-  }
-}
-
 // ------------------------------------------------------------------ post_reduce (plain)
 // Without equilibration only the three per-matrix sums are needed. For each 64-column
 // band of the super-tile the block handles two 32-row sub-tiles at a time and issues
@@ -421,6 +285,156 @@ __global__ void __launch_bounds__(kThreads, 4) post_reduce_plain_kernel(const El
   }
   const double xs = slab_scale(a, k);
   double acc[3] = {ww, wo * xs, oo * xs * xs};
+  block_sum<3>(acc, red);
+  if (threadIdx.x == 0) {
+    atomicAdd(&a.scal[k].w2, acc[0]);
+    atomicAdd(&a.scal[k].wo, acc[1]);
+    atomicAdd(&a.scal[k].o2, acc[2]);
+  }
+}
+
+// ------------------------------------------------------------------ post_reduce (equilibration)
+// Equilibration and the two-sided mode: the three per-matrix sums plus the per-row and
+// per-column sums of O^2 and W*O in the storage frame. Same walk and loads as the plain
+// reduction (two 32-row sub-tiles in flight per thread). Each thread keeps the sums of
+// its 8 columns over the band's rows and of its 4 rows over the super-tile in
+// registers; a band's column sums are reduced across the 4 rows of a warp by shuffles
+// and across the 8 warps through shared memory (double-buffered by band, one barrier
+// per band); the row sums are reduced across the 8 lanes of a row by shuffles at the
+// end. One atomic per row and per column of the super-tile. The slab scale multiplies
+// the finished sums.
+template <bool XF32>
+__global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  __shared__ float tile[kRedGroup][kTC][kTR + 1];
+  __shared__ float colred[2][2][kThreads / 32][kTC];  // [band parity][sum][warp][column]
+  __shared__ double red[3][kThreads / 32];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
+  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const bool vec = (d.flags & MAT_VEC_OK) != 0;
+  const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  const float xs = slab_scale(a, k);
+  float ww = 0.f, wo = 0.f, oo = 0.f;
+  float row_o2[kSubR], row_wo[kSubR];  // this thread's share of its 4 rows' sums
+#pragma unroll
+  for (int i = 0; i < kSubR; ++i) row_o2[i] = row_wo[i] = 0.f;
+
+  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {  // uniform over the block
+    const int c0 = C0 + bj * kTC;
+    float col_o2[8], col_wo[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) col_o2[e] = col_wo[e] = 0.f;
+#pragma unroll
+    for (int g0 = 0; g0 < kSubR; g0 += kRedGroup) {
+      if (R0 + g0 * kTR >= d.rows) break;  // uniform over the block
+      float w[kRedGroup][8], o[kRedGroup][8];
+#pragma unroll
+      for (int q = 0; q < kRedGroup; ++q) {
+        const int r0 = R0 + (g0 + q) * kTR;
+        const int r = r0 + lr, c = c0 + lc;
+        const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+        if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w[q]);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[q][e] = 0.f;
+        }
+        int64_t off;
+        int v2;
+        if (!tall) {
+          off = (int64_t)r * s.ldx + c;
+          v2 = valid;
+        } else {
+          const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
+          off = (int64_t)sr * s.ldx + sc;
+          v2 = (sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
+        }
+        if (v2 > 0) load8_slab(s.xf, XF32, off, v2, o[q]);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[q][e] = 0.f;
+        }
+      }
+      if (tall) {  // block-uniform
+#pragma unroll
+        for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) tile[q][threadIdx.x >> 2][(threadIdx.x & 3) * 8 + e] = o[q][e];
+        __syncthreads();
+#pragma unroll
+        for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[q][e] = tile[q][lc + e][lr];
+        __syncthreads();  // the tiles are reused by the next group
+      }
+#pragma unroll
+      for (int q = 0; q < kRedGroup; ++q)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {  // elements outside the matrix are 0 on both sides
+          const float o2 = o[q][e] * o[q][e], wov = w[q][e] * o[q][e];
+          ww = fmaf(w[q][e], w[q][e], ww);
+          wo += wov;
+          oo += o2;
+          row_o2[g0 + q] += o2;
+          row_wo[g0 + q] += wov;
+          col_o2[e] += o2;
+          col_wo[e] += wov;
+        }
+    }
+    // the band's column sums: the 4 rows of a warp share columns every 8 lanes
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+#pragma unroll
+      for (int m = 8; m < 32; m <<= 1) {
+        col_o2[e] += __shfl_xor_sync(0xffffffffu, col_o2[e], m);
+        col_wo[e] += __shfl_xor_sync(0xffffffffu, col_wo[e], m);
+      }
+    }
+    const int buf = bj & 1;
+    if (lane < 8) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        colred[buf][0][warp][lc + e] = col_o2[e];
+        colred[buf][1][warp][lc + e] = col_wo[e];
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < 2 * kTC) {
+      const int which = threadIdx.x / kTC, cc = threadIdx.x % kTC;
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < kThreads / 32; ++i) sum += colred[buf][which][i][cc];
+      if (c0 + cc < d.cols) {
+        if (which) atomicAdd(a.eq_wo + s.eq_off + d.rows + c0 + cc, sum * xs);
+        else atomicAdd(a.eq_o2 + s.eq_off + d.rows + c0 + cc, sum * xs * xs);
+      }
+    }
+    // the next band writes the other buffer; the band after it passes this band's
+    // barrier only once every thread has read this buffer
+  }
+  // row sums: the 8 threads of a row are consecutive lanes
+#pragma unroll
+  for (int bi = 0; bi < kSubR; ++bi) {
+    float ro = row_o2[bi], rw = row_wo[bi];
+#pragma unroll
+    for (int m = 4; m > 0; m >>= 1) {
+      ro += __shfl_xor_sync(0xffffffffu, ro, m);
+      rw += __shfl_xor_sync(0xffffffffu, rw, m);
+    }
+    const int r = R0 + bi * kTR + lr;
+    if ((threadIdx.x & 7) == 0 && r < d.rows) {
+      atomicAdd(a.eq_o2 + s.eq_off + r, ro * xs * xs);
+      atomicAdd(a.eq_wo + s.eq_off + r, rw * xs);
+    }
+  }
+  double acc[3] = {ww, (double)wo * xs, (double)oo * xs * xs};
   block_sum<3>(acc, red);
   if (threadIdx.x == 0) {
     atomicAdd(&a.scal[k].w2, acc[0]);
@@ -677,7 +691,9 @@ cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
 }
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
-  if (a.equilibrate) return launch_pdl(post_reduce_eq_kernel, a.total_tiles, s, a);
+  if (a.equilibrate)
+    return a.x_fp32 ? launch_pdl(post_reduce_eq_kernel<true>, a.total_tiles, s, a)
+                    : launch_pdl(post_reduce_eq_kernel<false>, a.total_tiles, s, a);
   return a.x_fp32 ? launch_pdl(post_reduce_plain_kernel<true>, a.total_tiles, s, a)
                   : launch_pdl(post_reduce_plain_kernel<false>, a.total_tiles, s, a);
 }

@@ -43,6 +43,10 @@ struct ClassMaps {
   CUtensorMap x32[2];   // output boxes of one epilogue warp: 64 x 32
   CUtensorMap s32;
   CUtensorMap p32;
+  // single-CTA symmetric phases load B in 64-row units
+  CUtensorMap x64[2];   // X slabs, 64 x 64 boxes
+  CUtensorMap s64;      // S slab, 64 x 64 boxes
+  CUtensorMap smir1;    // S slab, chunk view, one chunk
 };
 
 }  // namespace
@@ -81,6 +85,7 @@ struct muon_plan_s {
   // on a private stream; a failed capture leaves the plan eager for good.
   bool use_graph = false;
   bool graph_ok = true;
+  bool graph_stale = false;  // hyper-parameters changed: update the executable in place
   int eager_steps = 0;
   cudaGraphExec_t graph_exec = nullptr;
   void* graph_ws = nullptr;
@@ -90,6 +95,7 @@ struct muon_plan_s {
   void drop_graph() {
     if (graph_exec != nullptr) cudaGraphExecDestroy(graph_exec);
     graph_exec = nullptr;
+    graph_stale = false;
   }
   ~muon_plan_s() {
     for (const ProfRec& r : recs) {
@@ -413,7 +419,10 @@ muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t str
         ok = ok && encode_chunk_map_bf16(&cm.xmn[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx,
                                          ci.m % kPairTile == 0 ? 2 : tc_block_n(PH_APPLY) / 64);
         ok = ok && encode_slab_map_bf16(&cm.x32[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 32);
+        ok = ok && encode_slab_map_bf16(&cm.x64[b], base + ci.off_x[b], ci.n, ci.m, ci.count, ci.ldx, 64, 64);
       }
+      ok = ok && encode_slab_map_bf16(&cm.s64, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 64);
+      ok = ok && encode_chunk_map_bf16(&cm.smir1, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 1);
       ok = ok && encode_slab_map_bf16(&cm.s32, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 32);
       ok = ok && encode_slab_map_bf16(&cm.p32, base + ci.off_p, ci.m, ci.m, ci.count, ci.lds, 64, 32);
       ok = ok && encode_slab_map_bf16(&cm.s128, base + ci.off_s, ci.m, ci.m, ci.count, ci.lds, 64, 128);
@@ -439,8 +448,10 @@ muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t str
   return MUON_OK;
 }
 
+// var_sym: the single-CTA tensor-core kernel, whose symmetric phases cut each 128-row
+// block into variable-width pieces (sym_piece) instead of bn x bn tiles.
 void fill_class_args(const muon_plan_s* p, uint8_t* base, size_t c, int phase, int it,
-                     NsClassArgs* k, int bm, int bn, int bk) {
+                     NsClassArgs* k, int bm, int bn, int bk, bool var_sym = false) {
   const ClassInfo& ci = p->classes[c];
   const int esz = p->x_fp32 ? 4 : 2;
   k->m = ci.m;
@@ -459,6 +470,7 @@ void fill_class_args(const muon_plan_s* p, uint8_t* base, size_t c, int phase, i
   k->tiles_i = (ci.m + bm - 1) / bm;
   k->tiles_j = (ncols + bn - 1) / bn;
   k->tiles_per_mat = phase == PH_APPLY ? k->tiles_i * k->tiles_j : k->tiles_i * (k->tiles_i + 1) / 2;
+  if (var_sym && phase != PH_APPLY) k->tiles_per_mat = sym_tiles_per_matrix(ci.m);
   const int K = phase == PH_GRAM ? ci.n : ci.m;
   k->k_blocks = (K + bk - 1) / bk;
 }
@@ -630,22 +642,24 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
               const ClassMaps& cm = p->maps[cid];
               const int bm = pair ? kPairTile : tc_block_m();
               const int bn = pair ? kPairTile : tc_block_n(phase);
-              fill_class_args(p, base, cid, phase, it, &a.cls[c], bm, bn, tc_block_k());
+              fill_class_args(p, base, cid, phase, it, &a.cls[c], bm, bn, tc_block_k(), !pair);
               a.tile_base[c] = tiles;
               tiles += a.cls[c].count * a.cls[c].tiles_per_mat;
               fl += class_phase_flops(p->classes[cid], phase);
               // S and P' hold only their blocks on or above the (tile) diagonal; the
               // *_t maps fetch mirror blocks for the operands below it
+              // (single-CTA symmetric phases take B in 64-row units: 64 x 64 boxes or
+              // one-chunk mirrors)
               if (phase == PH_GRAM) {
                 P.ta[c] = P.ta_t[c] = cm.x128[it % 2];
-                P.tb[c] = P.tb_t[c] = cm.x128[it % 2];
+                P.tb[c] = P.tb_t[c] = pair ? cm.x128[it % 2] : cm.x64[it % 2];
                 P.tc[c] = cm.s128;
                 P.td[c] = cm.s32;
               } else if (phase == PH_POLY) {
                 P.ta[c] = cm.s128;
                 P.ta_t[c] = cm.smir;
-                P.tb[c] = cm.s128;
-                P.tb_t[c] = cm.smir;
+                P.tb[c] = pair ? cm.s128 : cm.s64;
+                P.tb_t[c] = pair ? cm.smir : cm.smir1;
                 P.tc[c] = cm.s128;
                 P.td[c] = cm.p32;
               } else {
@@ -686,8 +700,13 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
 }
 
 // Captures one step of a bound plan into a CUDA graph on the plan's private stream.
+// With an executable of the same launch sequence already instantiated (only scalar
+// kernel arguments changed, e.g. a learning-rate schedule), the executable is updated
+// in place (cudaGraphExecUpdate) instead of being instantiated again.
 muon_status_t capture_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int dev, int num_sms) {
-  p->drop_graph();
+  cudaGraphExec_t old_exec = p->graph_stale ? p->graph_exec : nullptr;
+  if (old_exec == nullptr) p->drop_graph();
+  p->graph_stale = false;
   if (p->cap_stream == nullptr &&
       cudaStreamCreateWithFlags(&p->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
     cudaGetLastError();
@@ -703,7 +722,20 @@ muon_status_t capture_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int de
   if (st != MUON_OK || e != cudaSuccess || graph == nullptr) {
     if (graph != nullptr) cudaGraphDestroy(graph);
     cudaGetLastError();
+    p->drop_graph();
     return MUON_ERR_CUDA;
+  }
+  if (old_exec != nullptr) {
+    cudaGraphExecUpdateResultInfo info;
+    if (cudaGraphExecUpdate(old_exec, graph, &info) == cudaSuccess) {
+      cudaGraphDestroy(graph);
+      p->graph_ws = ws;
+      p->graph_stats = stats;
+      p->graph_dev = dev;
+      return MUON_OK;  // same executable, new arguments
+    }
+    cudaGetLastError();
+    p->drop_graph();   // topology differs: instantiate afresh
   }
   cudaGraphExec_t exec = nullptr;
   const cudaError_t ei = cudaGraphInstantiate(&exec, graph, 0);
@@ -734,8 +766,8 @@ muon_status_t run_plan(muon_plan_s* p, void* ws, size_t ws_bytes, muon_stats_t* 
     if (st != MUON_OK) return st;
   }
   if (p->use_graph && p->graph_ok && !p->prof) {
-    const bool same = p->graph_exec != nullptr && p->graph_ws == ws && p->graph_stats == stats &&
-                      p->graph_dev == dev;
+    const bool same = p->graph_exec != nullptr && !p->graph_stale && p->graph_ws == ws &&
+                      p->graph_stats == stats && p->graph_dev == dev;
     if (!same && p->eager_steps > 0 && capture_step(p, ws, stats, dev, num_sms) != MUON_OK)
       p->graph_ok = false;  // stay eager
     if (p->graph_ok && p->graph_exec != nullptr && p->graph_ws == ws && p->graph_stats == stats &&
@@ -834,9 +866,14 @@ muon_status_t muon_plan_set_hparams(muon_plan_t plan, const muon_hparams_t* hp) 
   const int steps = hp->mode == MUON_MODE_TWOSIDED ? 0 : hp->ns_steps;
   if ((steps == 0) != (plan->ns_steps == 0)) return MUON_ERR_INVALID_ARG;
   const bool parity_changed = (steps % 2) != (plan->ns_steps % 2);
+  const bool same_launches = steps == plan->ns_steps && hp->mode == plan->hp.mode &&
+                             (hp->mode == MUON_MODE_MUON) == (plan->hp.mode == MUON_MODE_MUON);
   plan->hp = *hp;
   plan->ns_steps = steps;
-  plan->drop_graph();                             // the captured launches hold the old values
+  // the captured launches hold the old values: with the same launch sequence the next
+  // step updates the executable in place, otherwise it is captured afresh
+  if (same_launches && plan->graph_exec != nullptr) plan->graph_stale = true;
+  else plan->drop_graph();
   if (parity_changed) plan->ws_cached = nullptr;  // the result slab moved: re-upload
   return MUON_OK;
 }

@@ -229,6 +229,7 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
       k.tiles_i = (m + bm - 1) / bm;
       k.tiles_j = (ncols + bn - 1) / bn;
       k.tiles_per_mat = phase == PH_APPLY ? k.tiles_i * k.tiles_j : k.tiles_i * (k.tiles_i + 1) / 2;
+      if (!fp32 && !pair && phase != PH_APPLY) k.tiles_per_mat = sym_tiles_per_matrix(m);
       k.k_blocks = ((phase == PH_GRAM ? n : m) + bk - 1) / bk;
       a.tile_base[0] = 0;
       a.tile_base[1] = k.tiles_per_mat;
@@ -239,17 +240,22 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
       const void* x_in = k.x_in;
       bool ok = true;
       // S and P' hold only their blocks on or above the diagonal; *_t maps fetch mirrors
+      // (single-CTA symmetric phases take B in 64-row units: 64 x 64 boxes or
+      // one-chunk mirrors)
       if (phase == PH_GRAM) {
         ok = encode_slab_map_bf16(&P.ta[0], x_in, n, m, 1, ldx, 64, 128) &&
+             encode_slab_map_bf16(&P.tb[0], x_in, n, m, 1, ldx, 64, pair ? 128 : 64) &&
              encode_slab_map_bf16(&P.tc[0], k.s, m, m, 1, lds, 64, 128) &&
              encode_slab_map_bf16(&P.td[0], k.s, m, m, 1, lds, 64, 32);
-        P.ta_t[0] = P.tb[0] = P.tb_t[0] = P.ta[0];
+        P.ta_t[0] = P.ta[0];
+        P.tb_t[0] = P.tb[0];
       } else if (phase == PH_POLY) {
         ok = encode_slab_map_bf16(&P.ta[0], k.s, m, m, 1, lds, 64, 128) &&
              encode_chunk_map_bf16(&P.ta_t[0], k.s, m, m, 1, lds, 2) &&
+             encode_slab_map_bf16(&P.tb[0], k.s, m, m, 1, lds, 64, pair ? 128 : 64) &&
+             encode_chunk_map_bf16(&P.tb_t[0], k.s, m, m, 1, lds, pair ? 2 : 1) &&
              encode_slab_map_bf16(&P.td[0], k.p, m, m, 1, lds, 64, 32);
-        P.tb[0] = P.tc[0] = P.ta[0];
-        P.tb_t[0] = P.ta_t[0];
+        P.tc[0] = P.ta[0];
       } else {
         ok = encode_slab_map_bf16(&P.ta[0], k.p, m, m, 1, lds, 64, 128) &&
              encode_chunk_map_bf16(&P.ta_t[0], k.p, m, m, 1, lds, 2) &&

@@ -67,6 +67,14 @@ template <int BN, int PHASE, bool PAIR>
 struct TcCfg {
   static constexpr bool kSym = PHASE != PH_APPLY;         // symmetric (upper-block) output
   static constexpr bool kHasC = PHASE == PH_POLY;         // epilogue reads a C tile (S)
+  // single-CTA symmetric phases: variable-width tiles (one row block, one column piece
+  // of up to BN = 256 columns; see sym_piece), B loaded in 64-row units
+  static constexpr bool kVarN = !PAIR && kSym;
+  // POLY's C tile (S): staged through shared memory by TMA (CTA pairs), or, for the
+  // short-K single-CTA tiles, read by each epilogue thread from global memory (L2)
+  // into registers before it waits for the accumulator
+  static constexpr bool kCStaged = kHasC && !kVarN;
+  static constexpr bool kCRegs = kHasC && kVarN;
   static constexpr int kNCol = PAIR ? 256 : BN;            // accumulator columns per CTA
   static constexpr int kBRows = PAIR ? 128 : BN;           // B rows (or columns) per CTA
   static constexpr int kABytes = BM * BK * 2;
@@ -76,7 +84,7 @@ struct TcCfg {
   static constexpr int kChunksPerWarp = kNCol / 128;
   static constexpr int kEpiBufs = (PAIR && kChunksPerWarp >= 2) ? 2 : 1;  // per-warp box buffers
   static constexpr int kStagingBytes =
-      kHasC ? BM * kNCol * 2 : kEpiWarps * kEpiBufs * kWarpBoxBytes;  // C tile, or per-warp boxes
+      kCStaged ? BM * kNCol * 2 : kEpiWarps * kEpiBufs * kWarpBoxBytes;  // C tile, or per-warp boxes
   static constexpr int kBudget = 224 * 1024;
   static constexpr int kFit = (kBudget - kStagingBytes) / kStageBytes;
   static constexpr int kStages = kFit > 8 ? 8 : kFit;
@@ -89,19 +97,42 @@ struct TcCfg {
   static constexpr int kTileM = PAIR ? 256 : 128;          // output tile (cluster) rows
   static constexpr int kTileN = PAIR ? 256 : BN;           // output tile columns
   static_assert(kStages >= 3, "pipeline too shallow");
+  static_assert(!kVarN || BN == 256, "variable-width tiles are at most 256 columns");
 };
 
 struct TileJob {
   int c, mat, ti, tj;
+  int col0, nt;  // first output column and width (columns) of the tile
 };
 
-__device__ __forceinline__ TileJob decode(const NsPhaseArgs& p, int t, bool sym) {
+// Tile t of the launch: its class, matrix and output block. Symmetric phases walk the
+// upper block triangle: fixed square tiles (tile_n x tile_n, CTA pairs) or, with varn,
+// the variable-width pieces of each 128-row block (sym_piece).
+__device__ __forceinline__ TileJob decode(const NsPhaseArgs& p, int t, bool sym, bool varn,
+                                          int tile_n) {
   int c = 0;
   while (c + 1 < p.num_classes && t >= p.tile_base[c + 1]) ++c;
   const NsClassArgs& k = p.cls[c];
   const int u = t - p.tile_base[c];
   TileJob j;
   j.c = c;
+  if (varn) {
+    // A matrix's tiles stay consecutive (they run at the same time and share its operand
+    // rows in L2), but the order of its pieces is rotated by the matrix index: pieces
+    // differ in width, and without the rotation a CTA of the round-robin would take the
+    // same piece of every matrix whenever the CTA count is a multiple of the pieces
+    j.mat = u / k.tiles_per_mat;
+    int rem = (u - j.mat * k.tiles_per_mat + j.mat) % k.tiles_per_mat;
+    int ti = 0;
+    while (rem >= sym_pieces(k.m, ti)) {
+      rem -= sym_pieces(k.m, ti);
+      ++ti;
+    }
+    j.ti = ti;
+    j.tj = rem;
+    sym_piece(k.m, ti, rem, &j.col0, &j.nt);
+    return j;
+  }
   j.mat = u / k.tiles_per_mat;
   int rem = u - j.mat * k.tiles_per_mat;
   if (sym) {
@@ -116,7 +147,15 @@ __device__ __forceinline__ TileJob decode(const NsPhaseArgs& p, int t, bool sym)
     j.ti = rem / k.tiles_j;
     j.tj = rem - j.ti * k.tiles_j;
   }
+  j.col0 = j.tj * tile_n;
+  j.nt = tile_n;
   return j;
+}
+
+// Whether B unit u (64 rows starting at output column col0 + 64 u) of k-block kb lies
+// below the stored 128-block diagonal (variable-width symmetric tiles).
+__device__ __forceinline__ bool unit_mirrored(bool sym_operand, int col0, int u, int kb) {
+  return sym_operand && (kb * 64) / 128 < (col0 + 64 * u) / 128;
 }
 
 // Byte offset of element (r, c) of a 128-row tile staged as 64-column boxes with
@@ -155,12 +194,13 @@ template <int BN, int PHASE, bool PAIR>
 __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_constant__ TcParams P) {
   using C = TcCfg<BN, PHASE, PAIR>;
   constexpr bool SYM = C::kSym;
-  constexpr bool HAS_C = C::kHasC;
+  constexpr bool HAS_C = C::kCStaged;        // C tile staged in shared memory by TMA
+  constexpr bool C_REGS = C::kCRegs;         // C read into registers from global memory
   constexpr int S = C::kStages;
   constexpr bool A_SYM = PHASE != PH_GRAM;   // A is S (POLY) or P' (APPLY): upper blocks only
   constexpr bool B_SYM = PHASE == PH_POLY;   // B is S
   constexpr bool B_MN = PHASE == PH_APPLY;   // B is X read along its rows
-  static_assert(PAIR || !SYM || BN == BM, "single-CTA symmetric phases use square tiles");
+  constexpr bool VARN = C::kVarN;            // variable-width symmetric tiles (single CTA)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -224,10 +264,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
       long long q = 0;
       bool ok = true;
       for (int t = unit; t < total && ok; t += nunits) {
-        const TileJob j = decode(p, t, SYM);
+        const TileJob j = decode(p, t, SYM, VARN, C::kTileN);
         const int kb_n = p.cls[j.c].k_blocks;
         const int a_row0 = j.ti * C::kTileM + rank * 128;
-        const int b_row0 = j.tj * C::kTileN + rank * (PAIR ? 128 : 0);
+        const int b_row0 = j.col0 + rank * (PAIR ? 128 : 0);
         for (int kb = 0; kb < kb_n; ++kb) {
           const int s = static_cast<int>(q % S);
           const uint32_t par = static_cast<uint32_t>((q / S) & 1);
@@ -237,6 +277,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           }
           uint8_t* sa = smem + s * C::kStageBytes;
           uint8_t* sb = sa + C::kABytes;
+          if (VARN) {
+            // A: the row block's 128 rows; B: the tile's nt rows in 64-row units, each
+            // K-major (a 64 x 64 box) or, below the diagonal, its mirror (one chunk)
+            mbar_expect_tx(&full[s], C::kABytes + j.nt * (BK * 2));
+            load_k_block<false>(sa, &P.ta[j.c], &P.ta_t[j.c], &full[s], a_row0, kb, j.mat,
+                                below_diag(A_SYM, j.ti * C::kTileM, kb, C::kTileM));
+            for (int u = 0; u < j.nt / 64; ++u) {
+              uint8_t* dst = sb + u * (64 * BK * 2);
+              if (unit_mirrored(B_SYM, j.col0, u, kb))
+                tma_load_4d(dst, &P.tb_t[j.c], &full[s], 0, kb * BK, j.col0 / 64 + u, j.mat);
+              else
+                tma_load_3d(dst, &P.tb[j.c], &full[s], kb * BK, j.col0 + 64 * u, j.mat);
+            }
+            ++q;
+            continue;
+          }
           if (!PAIR || rank == 0) mbar_expect_tx(&full[s], (PAIR ? 2 : 1) * C::kStageBytes);
           load_k_block<PAIR>(sa, &P.ta[j.c], &P.ta_t[j.c], &full[s], a_row0, kb, j.mat,
                              below_diag(A_SYM, j.ti * C::kTileM, kb, C::kTileM));
@@ -273,10 +329,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
       int it = 0;
       bool ok = true;
       for (int t = unit; t < total && ok; t += nunits, ++it) {
-        const TileJob j = decode(p, t, SYM);
+        const TileJob j = decode(p, t, SYM, VARN, C::kTileN);
         const int kb_n = p.cls[j.c].k_blocks;
         const int a_row0 = j.ti * C::kTileM;  // the first CTA's rows decide for both
-        const int b_row0 = j.tj * C::kTileN;
+        const int b_row0 = j.col0;
         const int ab = it & 1;
         const uint32_t apar = static_cast<uint32_t>((it >> 1) & 1);
         if (!mbar_wait(&tempty[ab], apar ^ 1u, abort_flag)) {
@@ -293,6 +349,38 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
             break;
           }
           tc_fence_after();
+          if (VARN) {
+            // B's 64-row units switch from K-major to mirrored (MN-major) at most once
+            // along the tile (unit_mirrored is monotone in u): one MMA per run of units
+            // of the same layout, each writing its own accumulator columns
+            const bool a_t = below_diag(A_SYM, a_row0, kb, C::kTileM);
+            const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
+            const uint32_t sb = sa + C::kABytes;
+            const uint64_t ad0 = (a_t ? mnmaj_hi : kmaj_hi) | static_cast<uint64_t>((sa >> 4) & 0x3FFFu);
+            const uint64_t astep = a_t ? 128u : 2u;
+            const int nu = j.nt / 64;
+            int split = nu;  // first mirrored unit
+            for (int u = 0; u < nu; ++u)
+              if (unit_mirrored(B_SYM, j.col0, u, kb)) { split = u; break; }
+#pragma unroll
+            for (int run = 0; run < 2; ++run) {
+              const int u0 = run == 0 ? 0 : split, u1 = run == 0 ? split : nu;
+              if (u1 <= u0) continue;
+              const bool b_t = run == 1;
+              const uint32_t idesc = idesc_bf16_f32(128, 64 * (u1 - u0), b_t) |
+                                     (a_t ? (1u << 15) : 0u);
+              const uint32_t sbu = sb + static_cast<uint32_t>(u0 * (64 * BK * 2));
+              const uint64_t bd0 = (b_t ? mnmaj_hi : kmaj_hi) | static_cast<uint64_t>((sbu >> 4) & 0x3FFFu);
+              const uint64_t bstep = b_t ? 128u : 2u;
+#pragma unroll
+              for (int kk = 0; kk < BK / 16; ++kk)
+                umma_f16(d_tmem + static_cast<uint32_t>(u0 * 64), ad0 + astep * kk, bd0 + bstep * kk,
+                         idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
+            umma_commit(&empty[s]);
+            ++q;
+            continue;
+          }
           // one instruction serves both CTAs of a pair: the layout choice is made per
           // cluster tile (block size kTileM), identical for both halves
           const bool a_t = below_diag(A_SYM, a_row0, kb, C::kTileM);
@@ -351,11 +439,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
     int nstore = 0;                                           // boxes this warp has staged
     bool c_pending = false;
     if (HAS_C && leader && unit < total) {
-      const TileJob j = decode(p, unit, SYM);
-      mbar_expect_tx(cfull, C::kStagingBytes);
-#pragma unroll
-      for (int h = 0; h < C::kNCol / 64; ++h)
-        tma_load_3d(stg + h * (BM * 128), &P.tc[j.c], cfull, j.tj * C::kTileN + h * 64,
+      const TileJob j = decode(p, unit, SYM, VARN, C::kTileN);
+      mbar_expect_tx(cfull, static_cast<uint32_t>(j.nt * (BM * 2)));
+      for (int h = 0; h < j.nt / 64; ++h)
+        tma_load_3d(stg + h * (BM * 128), &P.tc[j.c], cfull, j.col0 + h * 64,
                     j.ti * C::kTileM + rank * 128, j.mat);
       c_pending = true;
     }
@@ -365,10 +452,29 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
     int it = 0;
     bool ok = true;
     for (int t = unit; t < total; t += nunits, ++it) {
-      const TileJob j = decode(p, t, SYM);
+      const TileJob j = decode(p, t, SYM, VARN, C::kTileN);
       const NsClassArgs& k = p.cls[j.c];
       const int ab = it & 1;
       const uint32_t apar = static_cast<uint32_t>((it >> 1) & 1);
+      // C in registers: this thread's row of S for each of the warp's (at most two)
+      // chunks, loaded before the accumulator wait so that the fetch overlaps the MMAs.
+      // Columns past m inside the last chunk are the slab's padding: they only reach
+      // output columns the store clips.
+      uint4 creg[C_REGS ? 2 : 1][8];
+      if (C_REGS && ok) {
+        const int row = j.ti * C::kTileM + quad * 32 + lane;
+        const uint16_t* srow = static_cast<const uint16_t*>(k.s) + j.mat * k.sstride +
+                               static_cast<int64_t>(row) * k.lds + j.col0;
+#pragma unroll
+        for (int ci = 0; ci < (C_REGS ? 2 : 1); ++ci) {
+          const int c64 = 2 * ci + grp;
+          const bool have = row < k.m && c64 < j.nt / 64;
+#pragma unroll
+          for (int q8 = 0; q8 < 8; ++q8)
+            creg[ci][q8] = have ? __ldg(reinterpret_cast<const uint4*>(srow + c64 * 64) + q8)
+                                : make_uint4(0, 0, 0, 0);
+        }
+      }
       bool okw = ok && __all_sync(0xffffffffu, mbar_wait(&tfull[ab], apar, abort_flag));
       if (okw && HAS_C) okw = __all_sync(0xffffffffu, mbar_wait(cfull, it & 1, abort_flag));
       if (!okw && ok) {
@@ -381,7 +487,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
       const int m = k.m;
       const int ncols = PHASE == PH_APPLY ? k.n : m;
       const int row0 = j.ti * C::kTileM + rank * 128;   // this CTA's first output row
-      const int col0 = j.tj * C::kTileN;                 // this CTA's first output column
+      const int col0 = j.col0;                           // this CTA's first output column
       if (ok) {
         if (leader) c_pending = false;
         tc_fence_after();
@@ -390,8 +496,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           const double inv = 1.0 / (sqrt(p.scal[k.first + j.mat].u2) + (double)p.eps);
           scale = static_cast<float>(PHASE == PH_GRAM ? inv * inv : inv);
         }
+        // this warp's chunks of the tile: grp, grp + 2, ... below nt / 64
+        const int nchw = VARN ? (j.nt / 64 - grp + 1) / 2 : C::kChunksPerWarp;
+        if (nchw == 0) {  // nothing to read: release the accumulator at once
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[ab]);
+        }
 #pragma unroll 1
-        for (int ci = 0; ci < C::kChunksPerWarp; ++ci) {
+        for (int ci = 0; ci < nchw; ++ci) {
           const int c64 = 2 * ci + grp;  // 64-column chunk of the tile
           uint32_t v[2][32];
           const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
@@ -399,7 +512,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           tmem_ld32(taddr, v[0]);
           tmem_ld32(taddr + 32, v[1]);
           tmem_wait_ld();
-          if (ci == C::kChunksPerWarp - 1) {
+          if (ci == nchw - 1) {
             // this warp has read its share of the accumulator: free it for the MMA
             tc_fence_before();
             __syncwarp();
@@ -411,7 +524,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           uint8_t* box;
           if (HAS_C) {
             box = stg + c64 * (BM * 128) + quad * kWarpBoxBytes;  // this warp's rows of C
-          } else {
+          } else {  // GRAM, APPLY, and POLY with C in registers
             box = wbuf + (nstore % C::kEpiBufs) * kWarpBoxBytes;
             if (nstore >= C::kEpiBufs) {  // the store that last read this buffer is done with it
               if (lane == 0) tma_store_wait_read_n<C::kEpiBufs - 1>();
@@ -425,6 +538,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
             const uint32_t off = sw128_off(lane, q8 * 8);
             uint4 cw = make_uint4(0, 0, 0, 0);
             if (HAS_C) cw = *reinterpret_cast<const uint4*>(box + off);
+            if (C_REGS) cw = ci == 0 ? creg[0][q8] : creg[C_REGS ? 1 : 0][q8];  // no dynamic index
             const uint32_t cwv[4] = {cw.x, cw.y, cw.z, cw.w};
             uint32_t pk[4];
 #pragma unroll
@@ -461,11 +575,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
         named_barrier(1, kEpiWarps * 32);
         const int tn = t + nunits;
         if (leader && ok && tn < total) {
-          const TileJob jn = decode(p, tn, SYM);
-          mbar_expect_tx(cfull, C::kStagingBytes);
-#pragma unroll
-          for (int b = 0; b < C::kNCol / 64; ++b)
-            tma_load_3d(stg + b * (BM * 128), &P.tc[jn.c], cfull, jn.tj * C::kTileN + b * 64,
+          const TileJob jn = decode(p, tn, SYM, VARN, C::kTileN);
+          mbar_expect_tx(cfull, static_cast<uint32_t>(jn.nt * (BM * 2)));
+          for (int b = 0; b < jn.nt / 64; ++b)
+            tma_load_3d(stg + b * (BM * 128), &P.tc[jn.c], cfull, jn.col0 + b * 64,
                         jn.ti * C::kTileM + rank * 128, jn.mat);
           c_pending = true;
         }
@@ -518,7 +631,7 @@ cudaError_t launch_tc(const TcParams& P, int grid, cudaStream_t s) {
 
 }  // namespace
 
-int tc_block_n(int phase) { return phase == PH_APPLY ? 256 : 128; }
+int tc_block_n(int phase) { return phase == PH_APPLY ? 256 : 128; }  // symmetric: pieces, see sym_piece
 int tc_block_m() { return BM; }
 int tc_block_k() { return BK; }
 
@@ -538,8 +651,8 @@ cudaError_t launch_ns_phase_tc(const TcParams& P, int num_sms, cudaStream_t s) {
   if (total <= 0) return cudaSuccess;
   const int grid = total < num_sms ? total : num_sms;
   switch (P.args.phase) {
-    case PH_GRAM: return launch_tc<128, PH_GRAM, false>(P, grid, s);
-    case PH_POLY: return launch_tc<128, PH_POLY, false>(P, grid, s);
+    case PH_GRAM: return launch_tc<256, PH_GRAM, false>(P, grid, s);
+    case PH_POLY: return launch_tc<256, PH_POLY, false>(P, grid, s);
     default: return launch_tc<256, PH_APPLY, false>(P, grid, s);
   }
 }

@@ -26,6 +26,32 @@ int tc_block_m();
 int tc_block_n(int phase);
 int tc_block_k();
 
+// Symmetric phases (GRAM, POLY) of single-CTA classes: the m x m output is stored as its
+// 128 x 128 blocks on or above the block diagonal. Row block i (rows 128 i ..) is cut into
+// column pieces from column 128 i to m, each at most 256 wide and a multiple of 64, of
+// nearly equal width; a tile is one (row block, piece) pair and the MMA N is the piece
+// width. The host counts tiles and the kernel decodes them with these same functions.
+__host__ __device__ inline int sym_row_blocks(int m) { return (m + 127) / 128; }
+__host__ __device__ inline int sym_pieces(int m, int i) { return (m - 128 * i + 255) / 256; }
+__host__ __device__ inline int sym_piece_width(int m, int i) {
+  const int len = m - 128 * i, np = (len + 255) / 256;
+  return ((len + np - 1) / np + 63) / 64 * 64;
+}
+// Column start and width (a multiple of 64; the last piece may reach past m, where the
+// stores are clipped) of piece j of row block i.
+__host__ __device__ inline void sym_piece(int m, int i, int j, int* col0, int* width) {
+  const int w = sym_piece_width(m, i);
+  const int c0 = 128 * i + j * w;
+  const int rest = (m - c0 + 63) / 64 * 64;
+  *col0 = c0;
+  *width = w < rest ? w : rest;
+}
+__host__ __device__ inline int sym_tiles_per_matrix(int m) {
+  int t = 0;
+  for (int i = 0; i < sym_row_blocks(m); ++i) t += sym_pieces(m, i);
+  return t;
+}
+
 cudaError_t launch_ns_phase_tc(const TcParams& P, int num_sms, cudaStream_t s);
 
 // CTA-pair launch: 256 x 256 tiles (tiles_i = ceil(m/256), tiles_j = ceil(cols/256)),

@@ -321,6 +321,42 @@ def test_plan_hparams_change_between_steps(env):
     plan.close()
 
 
+def test_plan_learning_rate_schedule_updates_the_graph(env):
+    """A new learning rate and decay before every step (muon_plan_set_hparams with the
+    same launch sequence): from the third step on the captured graph is updated in place
+    instead of re-instantiated. Every step against the oracle with that step's lr."""
+    B, torch = env
+    shapes = [(128, 256), (768, 512), (320, 512)]
+    W0 = [H.seeded(r, c, 1700 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded_bf16(r, c, 1800 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(6)]
+    lrs = [0.02, 0.015, 0.01, 0.03, 0.005, 0.02]
+    wds = [0.0, 0.1, 0.0, 0.05, 0.1, 0.0]
+    Ws = [torch.tensor(w, device="cuda") for w in W0]
+    Ms = [torch.zeros_like(w) for w in Ws]
+    Gs = [torch.empty(w.shape, dtype=torch.bfloat16, device="cuda") for w in Ws]
+    plan = B.Plan(Ws, Gs, Ms, H.gpu_hp(B, mode="muongs", lr=lrs[0]))
+    W_orc = [w.astype(np.float64) for w in W0]
+    M_orc = [np.zeros_like(w) for w in W_orc]
+    for t in range(6):
+        plan.set_hparams(H.gpu_hp(B, mode="muongs", lr=lrs[t], wd=wds[t]))
+        ohp = H.oracle_hp(mode="muongs", lr=lrs[t], wd=wds[t])
+        W_prev_gpu = [w.double().cpu().numpy() for w in Ws]
+        W_prev_orc = [w.copy() for w in W_orc]
+        for g_dev, g in zip(Gs, grads[t]):
+            g_dev.copy_(torch.from_numpy(np.ascontiguousarray(g, dtype=np.float32)))
+        plan.step()
+        torch.cuda.synchronize()
+        for i in range(len(shapes)):
+            r = orc.muon_step(W_orc[i], grads[t][i].astype(np.float64), M_orc[i], ohp)
+            W_orc[i], M_orc[i] = r.W, r.M
+            Wg = Ws[i].double().cpu().numpy()
+            assert H.rel(Wg, W_orc[i]) <= H.TOL_BF16, (t, i)
+            assert H.rel(W_prev_gpu[i] - Wg, W_prev_orc[i] - W_orc[i]) <= H.TOL_BF16, (t, i)
+    assert plan.query_device_status() == 0
+    plan.close()
+
+
 def test_plan_graph_replay_matches_eager_steps(env):
     """A cached plan runs its first step eagerly, captures the second into a CUDA graph
     and replays it afterwards (re-capturing when the stats pointer changes). Four plan

@@ -204,7 +204,8 @@ MUON_API muon_status_t muon_newton_schulz_batched(const muon_ns_matrix_t* mats, 
 
 /* ---- per-kernel device timing of a plan (CUDA events around each launch) ----
  * Kernel kinds: "ingest", "ns_gram", "ns_poly", "ns_apply", "post_reduce",
- * "post_finalize", "post_apply". flops / bytes are the algorithmic work of the
+ * "post_finalize", "post_apply", "ns_fused" (the fp32 path's single launch over all
+ * iterations of small matrices). flops / bytes are the algorithmic work of the
  * recorded launches: Newton-Schulz flops count the symmetric Gram and polynomial
  * once (m(m+1)n and m^2(m+1)) and the apply 2m^2n; bytes count each kernel's own
  * inputs and outputs once (ingest: G, M read, M and X_0 written; post_reduce: W and

@@ -29,8 +29,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kTR = 32;   // sub-tile rows
 constexpr int kTC = 64;   // sub-tile cols
-constexpr int kSubR = kElemTileR / kTR;  // 4 sub-tiles down a super-tile
-constexpr int kSubC = kElemTileC / kTC;  // 4 sub-tiles across
+constexpr int kSubR = kElemTileR / kTR;  // at most 4 sub-tiles down a super-tile
 
 __device__ __forceinline__ void load8_f32(const float* p, bool vec, int valid, float (&v)[8]) {
   if (vec && valid == 8) {
@@ -188,11 +187,12 @@ __global__ void __launch_bounds__(kThreads, 8) ingest_kernel(const ElemArgs a) {
   const DevMat d = a.mats[k];
   const DevSlab s = a.slabs[k];
   const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
-  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
+  const int sub_r = a.sub_r, sub_c = a.sub_c;  // 32-row / 64-column sub-tiles per super-tile
+  const int tiles_c = (d.cols + sub_c * kTC - 1) / (sub_c * kTC);
+  const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
   float sq = 0.f;
-  for (int bi = 0; bi < kSubR && R0 + bi * kTR < d.rows; ++bi)
-    for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj)
+  for (int bi = 0; bi < sub_r && R0 + bi * kTR < d.rows; ++bi)
+    for (int bj = 0; bj < sub_c && C0 + bj * kTC < d.cols; ++bj)
       sq += ingest_subtile(a, d, s, R0 + bi * kTR, C0 + bj * kTC, tile);
   double acc[1] = {sq};
   block_sum<1>(acc, red);
@@ -223,15 +223,16 @@ __global__ void __launch_bounds__(kThreads, 4) post_reduce_plain_kernel(const El
   const DevMat d = a.mats[k];
   const DevSlab s = a.slabs[k];
   const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
-  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
+  const int sub_r = a.sub_r, sub_c = a.sub_c;  // 32-row / 64-column sub-tiles per super-tile
+  const int tiles_c = (d.cols + sub_c * kTC - 1) / (sub_c * kTC);
+  const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
   float ww = 0.f, wo = 0.f, oo = 0.f;
-  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
+  for (int bj = 0; bj < sub_c && C0 + bj * kTC < d.cols; ++bj) {
     const int c0 = C0 + bj * kTC;
-    for (int g0 = 0; g0 < kSubR && R0 + g0 * kTR < d.rows; g0 += kRedGroup) {
+    for (int g0 = 0; g0 < sub_r && R0 + g0 * kTR < d.rows; g0 += kRedGroup) {
       float w[kRedGroup][8], o[kRedGroup][8];
       // loads: W in the storage frame; the slab in the storage frame (wide) or as
       // 64 x 32 tiles of O^T (tall: slab rows = storage columns)
@@ -239,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 4) post_reduce_plain_kernel(const El
       for (int q = 0; q < kRedGroup; ++q) {
         const int r0 = R0 + (g0 + q) * kTR;
         const int r = r0 + lr, c = c0 + lc;
-        const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+        const bool inq = g0 + q < sub_r;  // the group's second sub-tile may lie past the super-tile
+        const int valid = (inq && r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
         if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w[q]);
         else {
 #pragma unroll
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 4) post_reduce_plain_kernel(const El
         } else {
           const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
           off = (int64_t)sr * s.ldx + sc;
-          v2 = (sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
+          v2 = (inq && sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
         }
         if (v2 > 0) load8_slab(s.xf, XF32, off, v2, o[q]);
         else {
@@ -315,32 +317,34 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
   const DevMat d = a.mats[k];
   const DevSlab s = a.slabs[k];
   const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
-  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
+  const int sub_r = a.sub_r, sub_c = a.sub_c;  // 32-row / 64-column sub-tiles per super-tile
+  const int tiles_c = (d.cols + sub_c * kTC - 1) / (sub_c * kTC);
+  const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
   const float xs = slab_scale(a, k);
-  float ww = 0.f, wo = 0.f, oo = 0.f;
-  float row_o2[kSubR], row_wo[kSubR];  // this thread's share of its 4 rows' sums
+  float ww = 0.f;
+  float row_o2[kSubR], row_wo[kSubR];  // this thread's share of its (up to 4) rows' sums
 #pragma unroll
   for (int i = 0; i < kSubR; ++i) row_o2[i] = row_wo[i] = 0.f;
 
-  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {  // uniform over the block
+  for (int bj = 0; bj < sub_c && C0 + bj * kTC < d.cols; ++bj) {  // uniform over the block
     const int c0 = C0 + bj * kTC;
     float col_o2[8], col_wo[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) col_o2[e] = col_wo[e] = 0.f;
 #pragma unroll
     for (int g0 = 0; g0 < kSubR; g0 += kRedGroup) {
-      if (R0 + g0 * kTR >= d.rows) break;  // uniform over the block
+      if (g0 >= sub_r || R0 + g0 * kTR >= d.rows) break;  // uniform over the block
       float w[kRedGroup][8], o[kRedGroup][8];
 #pragma unroll
       for (int q = 0; q < kRedGroup; ++q) {
         const int r0 = R0 + (g0 + q) * kTR;
         const int r = r0 + lr, c = c0 + lc;
-        const int valid = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+        const bool inq = g0 + q < sub_r;  // the group's second sub-tile may lie past the super-tile
+        const int valid = (inq && r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
         if (valid > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid, w[q]);
         else {
 #pragma unroll
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
         } else {
           const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
           off = (int64_t)sr * s.ldx + sc;
-          v2 = (sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
+          v2 = (inq && sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
         }
         if (v2 > 0) load8_slab(s.xf, XF32, off, v2, o[q]);
         else {
@@ -380,8 +384,6 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
         for (int e = 0; e < 8; ++e) {  // elements outside the matrix are 0 on both sides
           const float o2 = o[q][e] * o[q][e], wov = w[q][e] * o[q][e];
           ww = fmaf(w[q][e], w[q][e], ww);
-          wo += wov;
-          oo += o2;
           row_o2[g0 + q] += o2;
           row_wo[g0 + q] += wov;
           col_o2[e] += o2;
@@ -419,17 +421,21 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
     // the next band writes the other buffer; the band after it passes this band's
     // barrier only once every thread has read this buffer
   }
-  // row sums: the 8 threads of a row are consecutive lanes
+  // row sums: the 8 threads of a row are consecutive lanes; their totals over the
+  // super-tile are the block's shares of <W,O> and ||O||^2
+  float wo = 0.f, oo = 0.f;
 #pragma unroll
   for (int bi = 0; bi < kSubR; ++bi) {
     float ro = row_o2[bi], rw = row_wo[bi];
+    wo += rw;
+    oo += ro;
 #pragma unroll
     for (int m = 4; m > 0; m >>= 1) {
       ro += __shfl_xor_sync(0xffffffffu, ro, m);
       rw += __shfl_xor_sync(0xffffffffu, rw, m);
     }
     const int r = R0 + bi * kTR + lr;
-    if ((threadIdx.x & 7) == 0 && r < d.rows) {
+    if ((threadIdx.x & 7) == 0 && bi < sub_r && r < d.rows) {
       atomicAdd(a.eq_o2 + s.eq_off + r, ro * xs * xs);
       atomicAdd(a.eq_wo + s.eq_off + r, rw * xs);
     }
@@ -584,8 +590,9 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs 
   const DevMat d = a.mats[k];
   const DevSlab s = a.slabs[k];
   const int t = b - a.tile_prefix[k];
-  const int tiles_c = (d.cols + kElemTileC - 1) / kElemTileC;
-  const int R0 = (t / tiles_c) * kElemTileR, C0 = (t % tiles_c) * kElemTileC;
+  const int sub_r = a.sub_r, sub_c = a.sub_c;  // 32-row / 64-column sub-tiles per super-tile
+  const int tiles_c = (d.cols + sub_c * kTC - 1) / (sub_c * kTC);
+  const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
@@ -595,17 +602,18 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs 
   cf.cw = cf.co = 0.f;
   cf.axis = 0;
   if (!ns_only) cf = a.coef[k];
-  for (int bj = 0; bj < kSubC && C0 + bj * kTC < d.cols; ++bj) {
+  for (int bj = 0; bj < sub_c && C0 + bj * kTC < d.cols; ++bj) {
     const int c0 = C0 + bj * kTC;
     const int c = c0 + lc;
-    for (int g0 = 0; g0 < kSubR && R0 + g0 * kTR < d.rows; g0 += kRedGroup) {
+    for (int g0 = 0; g0 < sub_r && R0 + g0 * kTR < d.rows; g0 += kRedGroup) {
       float w[kRedGroup][8], o[kRedGroup][8];
       int valid[kRedGroup];
 #pragma unroll
       for (int q = 0; q < kRedGroup; ++q) {
         const int r0 = R0 + (g0 + q) * kTR;
         const int r = r0 + lr;
-        valid[q] = (r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
+        const bool inq = g0 + q < sub_r;  // the group's second sub-tile may lie past the super-tile
+        valid[q] = (inq && r < d.rows) ? max(0, min(8, d.cols - c)) : 0;
         if (!ns_only && valid[q] > 0) load8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid[q], w[q]);
         else {
 #pragma unroll
@@ -619,7 +627,7 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs 
         } else {
           const int sr = c0 + (threadIdx.x >> 2), sc = r0 + (threadIdx.x & 3) * 8;
           off = (int64_t)sr * s.ldx + sc;
-          v2 = (sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
+          v2 = (inq && sr < d.cols) ? max(0, min(8, d.rows - sc)) : 0;
         }
         if (v2 > 0) load8_slab(s.xf, XF32, off, v2, o[q]);
         else {

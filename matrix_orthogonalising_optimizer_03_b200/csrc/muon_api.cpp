@@ -63,6 +63,7 @@ struct muon_plan_s {
   std::vector<int64_t> eq_off;     // plan order
   std::vector<int32_t> tile_prefix;
   int64_t eq_total = 0;
+  int sub_r = 4, sub_c = 4;  // elementwise super-tile in 32 x 64 sub-tiles
   size_t off_scal = 0, off_coef = 0, off_desc = 0, off_slabs = 0, off_tiles = 0;
   size_t off_eq_o2 = 0, off_eq_wo = 0, ws_bytes = 0;
   // cached per workspace pointer and device
@@ -253,11 +254,15 @@ void build_plan(muon_plan_s* p) {
   p->dev.swap(sorted);
   p->eq_off.swap(eq_off);
   p->eq_total = p->equilibrate ? eq_total : 0;
-  // elementwise tiles
+  // elementwise tiles: one-sub-tile super-tiles for small steps, 128 x 256 otherwise
+  int64_t elems = 0;
+  for (int i = 0; i < n; ++i) elems += int64_t(p->dev[i].rows) * p->dev[i].cols;
+  p->sub_r = elems <= kElemSmallStep ? 1 : kElemTileR / kElemSubR;
+  p->sub_c = elems <= kElemSmallStep ? 1 : kElemTileC / kElemSubC;
+  const int tr = p->sub_r * kElemSubR, tc = p->sub_c * kElemSubC;
   p->tile_prefix.assign(n + 1, 0);
   for (int i = 0; i < n; ++i) {
-    const int64_t t = int64_t((p->dev[i].rows + kElemTileR - 1) / kElemTileR) *
-                      ((p->dev[i].cols + kElemTileC - 1) / kElemTileC);
+    const int64_t t = int64_t((p->dev[i].rows + tr - 1) / tr) * ((p->dev[i].cols + tc - 1) / tc);
     p->tile_prefix[i + 1] = static_cast<int32_t>(p->tile_prefix[i] + t);
   }
   // workspace layout
@@ -475,9 +480,11 @@ void fill_class_args(const muon_plan_s* p, uint8_t* base, size_t c, int phase, i
   k->k_blocks = (K + bk - 1) / bk;
 }
 
-enum ProfKind { PK_INGEST = 0, PK_GRAM, PK_POLY, PK_APPLY, PK_REDUCE, PK_FINALIZE, PK_POST, PK_COUNT };
+enum ProfKind { PK_INGEST = 0, PK_GRAM, PK_POLY, PK_APPLY, PK_REDUCE, PK_FINALIZE, PK_POST,
+                PK_NS_FUSED, PK_COUNT };
 const char* const kProfNames[PK_COUNT] = {"ingest", "ns_gram", "ns_poly", "ns_apply",
-                                          "post_reduce", "post_finalize", "post_apply"};
+                                          "post_reduce", "post_finalize", "post_apply",
+                                          "ns_fused"};
 constexpr size_t kMaxProfRecs = 1 << 16;
 
 cudaEvent_t prof_event(muon_plan_s* p) {
@@ -576,6 +583,8 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
   ea.x_fp32 = p->x_fp32 ? 1 : 0;
   ea.equilibrate = p->equilibrate ? 1 : 0;
   ea.xs_from_u2 = p->ns_steps == 0 ? 1 : 0;
+  ea.sub_r = p->sub_r;
+  ea.sub_c = p->sub_c;
 
   {
     ProfScope ps(p, stream);
@@ -585,10 +594,41 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
 
   // Newton-Schulz phases, at most kMaxClassesPerLaunch classes per launch
   const int nc = static_cast<int>(p->classes.size());
+  // fp32 path: small classes run every iteration in one fused launch; the others take
+  // one launch per phase
+  std::vector<int> fp32_small, fp32_large;
+  for (int c = 0; p->x_fp32 && c < nc; ++c)
+    (simt_fused_fits(p->classes[c].m, p->classes[c].n) ? fp32_small : fp32_large).push_back(c);
+  for (size_t g0 = 0; p->ns_steps > 0 && g0 < fp32_small.size(); g0 += kMaxClassesPerLaunch) {
+    const int cn = static_cast<int>(std::min<size_t>(kMaxClassesPerLaunch, fp32_small.size() - g0));
+    NsFusedArgs a{};
+    a.num_classes = cn;
+    a.steps = p->ns_steps;
+    a.a = hp.ns_coeffs[0];
+    a.b = hp.ns_coeffs[1];
+    a.c = hp.ns_coeffs[2];
+    a.eps = hp.eps;
+    a.scal = ea.scal;
+    int mats = 0;
+    double fl = 0;
+    for (int c = 0; c < cn; ++c) {
+      const int cid = fp32_small[g0 + c];
+      fill_class_args(p, base, cid, PH_GRAM, 0, &a.cls[c], 32, 32, 16);
+      a.x0[c] = base + p->classes[cid].off_x[0];
+      a.x1[c] = base + p->classes[cid].off_x[1];
+      a.mat_base[c] = mats;
+      mats += a.cls[c].count;
+      for (int ph = PH_GRAM; ph <= PH_APPLY; ++ph) fl += p->ns_steps * class_phase_flops(p->classes[cid], ph);
+    }
+    a.mat_base[cn] = mats;
+    ProfScope ps(p, stream);
+    if (launch_ns_simt_fused(a, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    ps.done(PK_NS_FUSED, fl, 0.0);
+  }
   for (int it = 0; it < p->ns_steps; ++it) {
     for (int phase = PH_GRAM; phase <= PH_APPLY; ++phase) {
-      for (int c0 = 0; p->x_fp32 && c0 < nc; c0 += kMaxClassesPerLaunch) {
-        const int cn = std::min(kMaxClassesPerLaunch, nc - c0);
+      for (size_t g0 = 0; g0 < fp32_large.size(); g0 += kMaxClassesPerLaunch) {
+        const int cn = static_cast<int>(std::min<size_t>(kMaxClassesPerLaunch, fp32_large.size() - g0));
         {
           NsPhaseArgs a{};
           a.num_classes = cn;
@@ -602,7 +642,7 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
           a.err = ea.err;
           int tiles = 0;
           for (int c = 0; c < cn; ++c) {
-            fill_class_args(p, base, c0 + c, phase, it, &a.cls[c], 64, 64, 16);
+            fill_class_args(p, base, fp32_large[g0 + c], phase, it, &a.cls[c], 64, 64, 16);
             a.tile_base[c] = tiles;
             tiles += a.cls[c].count * a.cls[c].tiles_per_mat;
           }
@@ -610,7 +650,7 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
           ProfScope ps(p, stream);
           if (launch_ns_phase_simt(a, stream) != cudaSuccess) return MUON_ERR_CUDA;
           double fl = 0;
-          for (int c = 0; c < cn; ++c) fl += class_phase_flops(p->classes[c0 + c], phase);
+          for (int c = 0; c < cn; ++c) fl += class_phase_flops(p->classes[fp32_large[g0 + c]], phase);
           ps.done(PK_GRAM + phase, fl, 0.0);
         }
       }

@@ -53,8 +53,13 @@ struct ClassInfo {
 };
 
 constexpr int kMaxClassesPerLaunch = 4;
-constexpr int kElemTileR = 128;  // elementwise super-tile: rows (storage frame)
-constexpr int kElemTileC = 256;  // elementwise super-tile: cols
+constexpr int kElemTileR = 128;  // largest elementwise super-tile: rows (storage frame)
+constexpr int kElemTileC = 256;  // largest elementwise super-tile: cols
+constexpr int kElemSubR = 32;    // elementwise sub-tile: rows
+constexpr int kElemSubC = 64;    // elementwise sub-tile: cols
+// Small steps (at most this many elements over all matrices) use one-sub-tile
+// super-tiles, so that more blocks share the work; larger ones use 128 x 256.
+constexpr int64_t kElemSmallStep = int64_t(1) << 22;
 
 // Workspace header: the sticky device error word and a step counter.
 struct WsHeader {
@@ -101,6 +106,7 @@ struct ElemArgs {
   int32_t x_fp32;       // slabs hold fp32 (else bf16)
   int32_t equilibrate;
   int32_t xs_from_u2;   // ns_steps == 0: the slab holds U, scale it by 1/(||U||+eps)
+  int32_t sub_r, sub_c; // super-tile = sub_r x sub_c sub-tiles of 32 x 64 (1..4 each)
 };
 
 cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s);
@@ -142,5 +148,25 @@ struct NsPhaseArgs {
 };
 
 cudaError_t launch_ns_phase_simt(const NsPhaseArgs& a, cudaStream_t s);
+
+// All iterations of the fp32 Newton-Schulz of small matrices in one launch (one
+// 8-block cluster per matrix). cls[c] describes class c; x0 / x1 are its two X slabs
+// (the iteration reads x0 on even and x1 on odd iterations); mat_base[c] is the first
+// launch-local matrix of class c.
+struct NsFusedArgs {
+  NsClassArgs cls[kMaxClassesPerLaunch];
+  void* x0[kMaxClassesPerLaunch];
+  void* x1[kMaxClassesPerLaunch];
+  int32_t mat_base[kMaxClassesPerLaunch + 1];
+  int32_t num_classes;
+  int32_t steps;
+  float a, b, c;
+  float eps;
+  const MatScalars* scal;
+};
+// Whether a class of the fp32 path (oriented m x n, m <= n) takes the fused kernel:
+// n <= 256, so that a tile's full-K operand panels fit in shared memory.
+bool simt_fused_fits(int m, int n);
+cudaError_t launch_ns_simt_fused(const NsFusedArgs& a, cudaStream_t s);
 
 }  // namespace muon

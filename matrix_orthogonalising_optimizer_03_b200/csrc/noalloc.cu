@@ -173,7 +173,11 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
   sl.eq_off = 0;
   sl.ldx = ldx;
   sl.cls = 0;
-  const int64_t tiles = ((rows + kElemTileR - 1) / kElemTileR) * ((cols + kElemTileC - 1) / kElemTileC);
+  // elementwise super-tiles as the batched path picks them for a one-matrix step
+  const bool small = rows * cols <= kElemSmallStep;
+  const int sub_r = small ? 1 : kElemTileR / kElemSubR, sub_c = small ? 1 : kElemTileC / kElemSubC;
+  const int64_t tiles = ((rows + sub_r * kElemSubR - 1) / (sub_r * kElemSubR)) *
+                        ((cols + sub_c * kElemSubC - 1) / (sub_c * kElemSubC));
   noalloc_setup_kernel<<<1, 32, 0, s>>>(base, d, sl, static_cast<int32_t>(tiles), status_dev);
   if (cudaGetLastError() != cudaSuccess) return MUON_ERR_CUDA;
 
@@ -190,6 +194,8 @@ extern "C" MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matri
   ea.ns_only = 1;
   ea.x_fp32 = fp32 ? 1 : 0;
   ea.xs_from_u2 = iterate ? 0 : 1;
+  ea.sub_r = sub_r;
+  ea.sub_c = sub_c;
   if (launch_ingest(ea, s) != cudaSuccess) return MUON_ERR_CUDA;
 
   // the same kernels and tile shapes the batched path picks for this shape: CTA

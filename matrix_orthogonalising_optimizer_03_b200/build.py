@@ -21,7 +21,7 @@ BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmuon.so")
 
 SOURCES = ["muon_api.cpp", "elementwise.cu", "ns_simt.cu", "ns_tc.cu", "noalloc.cu", "diagnostics.cu", "qkclip.cu"]
-HEADERS = ["muon_internal.h", "ptx.cuh", "ns_tc.h", "validate.h"]
+HEADERS = ["muon_internal.h", "elementwise.h", "ptx.cuh", "ns_tc.h", "validate.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",

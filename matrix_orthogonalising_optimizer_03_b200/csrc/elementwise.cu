@@ -21,6 +21,7 @@
 #include <cuda_runtime.h>
 
 #include "muon_internal.h"
+#include "elementwise.h"
 #include "ptx.cuh"
 
 namespace muon {

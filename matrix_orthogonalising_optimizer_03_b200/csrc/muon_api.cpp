@@ -19,6 +19,7 @@
 
 #include "muon.h"
 #include "muon_internal.h"
+#include "elementwise.h"
 #include "ns_tc.h"
 #include "validate.h"
 

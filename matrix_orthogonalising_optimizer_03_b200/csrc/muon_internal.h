@@ -84,35 +84,7 @@ struct DevSlab {
 };
 static_assert(sizeof(DevSlab) == 32, "DevSlab is 32 bytes");
 
-// Arguments of the memory-bound kernels.
-struct ElemArgs {
-  const DevMat* mats;
-  const DevSlab* slabs;
-  const int32_t* tile_prefix;  // n+1 entries: first elementwise tile of each matrix
-  int32_t n;
-  int32_t total_tiles;
-  MatScalars* scal;
-  MatCoef* coef;
-  float* eq_o2;     // per-row / per-column sums of O^2 (then equilibration factors)
-  float* eq_wo;     // per-row / per-column sums of W*O
-  muon_stats_t* stats;
-  uint32_t* err;
-  float mu;
-  float lr, wd, eps, scale_k;
-  int32_t scale_rule;
-  int32_t mode;
-  int32_t nesterov;
-  int32_t ns_only;      // X in / O out instead of the optimizer step
-  int32_t x_fp32;       // slabs hold fp32 (else bf16)
-  int32_t equilibrate;
-  int32_t xs_from_u2;   // ns_steps == 0: the slab holds U, scale it by 1/(||U||+eps)
-  int32_t sub_r, sub_c; // super-tile = sub_r x sub_c sub-tiles of 32 x 64 (1..4 each)
-};
 
-cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s);
-cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s);
-cudaError_t launch_post_finalize(const ElemArgs& a, cudaStream_t s);
-cudaError_t launch_post_apply(const ElemArgs& a, cudaStream_t s);
 
 }  // namespace muon
 
@@ -150,7 +122,7 @@ struct NsPhaseArgs {
 cudaError_t launch_ns_phase_simt(const NsPhaseArgs& a, cudaStream_t s);
 
 // All iterations of the fp32 Newton-Schulz of small matrices in one launch (one
-// 8-block cluster per matrix). cls[c] describes class c; x0 / x1 are its two X slabs
+// cluster of 16, or 8, blocks per matrix). cls[c] describes class c; x0 / x1 are its two X slabs
 // (the iteration reads x0 on even and x1 on odd iterations); mat_base[c] is the first
 // launch-local matrix of class c.
 struct NsFusedArgs {

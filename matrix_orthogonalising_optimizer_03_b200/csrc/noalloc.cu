@@ -27,6 +27,7 @@
 
 #include "muon.h"
 #include "muon_internal.h"
+#include "elementwise.h"
 #include "ns_tc.h"
 #include "validate.h"
 

@@ -57,7 +57,33 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--slice-every", type=int, default=1,
+                    help="profiling: keep every k-th matrix of the shape set (all classes in proportion)")
+    ap.add_argument("--slice-class", type=int, default=-1,
+                    help="profiling: keep only shape class i (in order of first appearance)")
+    ap.add_argument("--slice-count", type=int, default=0,
+                    help="profiling: with --slice-class, keep its first n matrices")
     return ap.parse_args()
+
+
+def sliced(w, args):
+    """The matrices of shape set w that a profiling slice keeps (all of them by default)."""
+    specs = w.matrices()
+    if args.slice_every > 1:
+        specs = [s for s in specs if s.index % args.slice_every == 0]
+    if args.slice_class >= 0:
+        shapes = []
+        for s in specs:
+            if (s.rows, s.cols) not in shapes:
+                shapes.append((s.rows, s.cols))
+        specs = [s for s in specs if (s.rows, s.cols) == shapes[args.slice_class]]
+        if args.slice_count > 0:
+            specs = specs[:args.slice_count]
+    return specs
+
+
+def is_sliced(args) -> bool:
+    return args.slice_every > 1 or args.slice_class >= 0
 
 
 def load_peaks():
@@ -348,12 +374,14 @@ def elementwise_rates(prof, peaks):
     return out
 
 
-def ns_rates(prof, w, steps: int, ms_total: float, peaks):
+def ns_rates(prof, w, steps: int, ms_total: float, peaks, specs=None):
     """Newton-Schulz throughput in algorithmic flops (symmetric Gram and polynomial
     counted once), over the whole step time and over the summed time of the
     Newton-Schulz launches, each as a fraction of the burst and sustained bf16 peaks."""
     from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
-    flops = wl.workload_ns_flops(w) * steps
+    per_step = (wl.workload_ns_flops(w) if specs is None
+                else sum(wl.ns_flops(s.rows, s.cols) for s in specs))
+    flops = per_step * steps
     ns_ms = sum(v["total_ms"] for k, v in prof.items() if k.startswith("ns_"))
     step_tf = flops / (ms_total / 1e3) / 1e12
     phase_tf = flops / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
@@ -368,15 +396,18 @@ def ns_rates(prof, w, steps: int, ms_total: float, peaks):
 
 
 # ------------------------------------------------------------------ one shape set on one GPU
-def set_inputs(w, dev, seed: int):
-    """Resident inputs of a shape set: W (fp32), M (fp32, zero) and one flat gradient
-    buffer with a view per matrix, drawn on the device (seeded)."""
+def set_inputs(w, dev, seed: int, specs=None):
+    """Resident inputs of a shape set (or of the matrices `specs` of it): W (fp32), M
+    (fp32, zero) and one flat gradient buffer with a view per matrix, drawn on the
+    device (seeded)."""
     import torch
     from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
-    specs = w.matrices()
+    all_specs = w.matrices()
+    specs = all_specs if specs is None else specs
     gdt = torch.bfloat16 if w.grad_dtype == "bf16" else torch.float32
     numel = sum(s.rows * s.cols for s in specs)
-    Ws, G_src = wl.device_inputs(w, dev, seed=seed)
+    subset = None if len(specs) == len(all_specs) else {s.index for s in specs}
+    Ws, G_src = wl.device_inputs(w, dev, seed=seed, only=subset)
     g_flat = torch.empty(numel, dtype=gdt, device=dev)
     Ms, Gs = [], []
     off = 0
@@ -413,13 +444,14 @@ def time_steps(step, steps: int, world: int, dev, stream, after_start=None):
     return rank_max(e0.elapsed_time(e1), world, dev)
 
 
-def measure_plan(B, w, run, args, dev, world: int, peaks, peak_src, seed: int, full: bool):
-    """The plain plan step of one shape set: warm-up, K timed steps, K profiled steps
-    (per-kernel CUDA events), and with `full` the end-to-end feed. Returns a summary
-    dict and the live objects the caller may reuse (weights, momenta, plan)."""
+def measure_plan(B, w, run, args, dev, world: int, peaks, peak_src, seed: int, full: bool,
+                 specs=None):
+    """The plain plan step of one shape set (or of the matrices `specs` of it): warm-up,
+    K timed steps, K profiled steps (per-kernel CUDA events), and with `full` the
+    end-to-end feed. Returns a summary dict and the live weights and momenta."""
     import torch
     from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
-    Ws, Gs, Ms, g_flat, numel, gdt = set_inputs(w, dev, seed)
+    Ws, Gs, Ms, g_flat, numel, gdt = set_inputs(w, dev, seed, specs)
     gsz = 2 if w.grad_dtype == "bf16" else 4
     hp = B.hparams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
                    equilibrate=run.equilibrate, ns_fp32=w.ns_fp32)
@@ -446,11 +478,14 @@ def measure_plan(B, w, run, args, dev, world: int, peaks, peak_src, seed: int, f
     launches = sum(p["launches"] for p in prof.values())
     out = {
         "value": throughput(args.steps, world, ms, "weak"), "unit": "steps/s",
-        "ms_per_step": ms / args.steps, "matrices": w.n_matrices, "params": w.n_params,
+        "ms_per_step": ms / args.steps,
+        "matrices": w.n_matrices if specs is None else len(specs),
+        "params": w.n_params if specs is None else sum(s.rows * s.cols for s in specs),
         "mode": run.mode, "weight_decay": run.weight_decay, "equilibrate": run.equilibrate,
         "ns_path": "fp32 CUDA cores" if w.ns_fp32 else "bf16 tcgen05",
-        **ns_rates(prof, w, args.steps, ms, peaks),
-        "roofline": roofline(prof, w, peaks, peak_src, w.name, ms),
+        **ns_rates(prof, w, args.steps, ms, peaks, specs),
+        "roofline": roofline(prof, w, peaks, peak_src, w.name if specs is None else None, ms,
+                             clocks),
         "elementwise": elementwise_rates(prof, peaks),
         "kernels": {k: {"launches_per_step": v["launches"] / args.steps,
                         "ms_per_step": v["total_ms"] / args.steps} for k, v in prof.items()
@@ -552,7 +587,7 @@ def measure_sharded(B, w, run, args, dev, world: int, rank: int, peaks, peak_src
            "gpu_launches_max_rank": int(round(launches)),
            "clocks": clocks}
     if prof:
-        out["roofline"] = roofline(prof, w, peaks, peak_src, w.name, ms)
+        out["roofline"] = roofline(prof, w, peaks, peak_src, w.name, ms, clocks)
     if e2e:
         # end to end: each step copies this rank's local gradients from pinned host
         # memory (on the compute stream, not overlapped) and reads the statistics back
@@ -612,6 +647,17 @@ def main():
     sharded_job = world > 1 and args.dist == "sharded"
     gsz = 2 if w.grad_dtype == "bf16" else 4
 
+    if is_sliced(args):
+        # a profiling slice of the shape set: the plan step only, no comparison legs
+        if world != 1:
+            raise SystemExit("profiling slices run on one GPU")
+        specs = sliced(w, args)
+        res, _, _ = measure_plan(B, w, run, args, dev, 1, peaks, peak_src, 0, full=False,
+                                 specs=specs)
+        print(json.dumps({"profiling_slice": {"workload": w.name, "every": args.slice_every,
+                                              "class": args.slice_class, "count": len(specs)},
+                          **res}), flush=True)
+        return 0
     if sharded_job:
         res = measure_sharded(B, w, run, args, dev, world, rank, peaks, peak_src, 0, e2e=True)
         line_core = {"value": res["value"], "ms_per_step": res["ms_per_step"],
@@ -658,7 +704,6 @@ def main():
                 ws = wl.WORKLOADS[name]
                 r, _, _ = measure_plan(B, ws, ws.runs[ridx], args, dev, 1, peaks, peak_src, 0,
                                        full=False)
-                r.pop("kernels", None)
                 per[f"{name}/{ws.runs[ridx].mode}" + ("+wd" if ws.runs[ridx].weight_decay else "")] = r
                 torch.cuda.empty_cache()
             extra["per_set"] = per
@@ -712,7 +757,7 @@ def plan_profile(B, plan):
                                     "flops": arr[i].flops, "bytes": arr[i].bytes} for i in range(n)}
 
 
-def roofline(prof, w, peaks, peak_src, workload, region_ms: float):
+def roofline(prof, w, peaks, peak_src, workload, region_ms: float, clocks=None):
     ns = {k: v for k, v in prof.items() if k.startswith("ns_") and v["launches"]}
     if not ns:
         return None
@@ -725,15 +770,20 @@ def roofline(prof, w, peaks, peak_src, workload, region_ms: float):
         return {"bound": "alu", "kernel": name, "achieved": achieved, "unit": "TFLOP/s",
                 "peak": alu_peak, "frac": achieved / alu_peak, "traffic": None,
                 "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flops x 1965 MHz"}
-    # a kernel inside a timed region of a second or more runs under the power cap:
-    # compare it with the sustained figure, a shorter region with the burst figure
-    sustained = region_ms >= 1000.0
+    # a kernel that ran under the power cap (the clock record shows sw_power_cap), or
+    # inside a timed region of a second or more, is in the sustained regime: compare it
+    # with the sustained figure; otherwise with the burst figure. Both are reported.
+    capped = clocks is not None and "sw_power_cap" in (clocks.get("reasons") or [])
+    sustained = region_ms >= 1000.0 or capped
     peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
     traffic = traffic_record(name, workload)
     return {"bound": "tensor", "kernel": name, "achieved": achieved, "peak": peak,
             "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+            "frac_burst": achieved / peaks["bf16_tflops"],
+            "frac_sustained": achieved / peaks["bf16_tflops_sustained"],
             "flops_per_launch": flops, "launch_ms": per_launch_s * 1e3,
-            "peak_source": f"{peak_src} bf16 ({'sustained' if sustained else 'burst'})"}
+            "peak_source": f"{peak_src} bf16 ({'sustained' if sustained else 'burst'}"
+                           f"{': sw_power_cap in the timed region' if capped else ''})"}
 
 
 if __name__ == "__main__":

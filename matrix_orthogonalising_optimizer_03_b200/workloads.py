@@ -164,14 +164,16 @@ def normal(rows: int, cols: int, seed: int, std: float, bf16: bool = False) -> n
     return bf16_round(x) if bf16 else x
 
 
-def device_inputs(w: Workload, device, seed: int = 0, exact=(), step: int = 0):
+def device_inputs(w: Workload, device, seed: int = 0, exact=(), step: int = 0, only=None):
     """W_0 and G_step for every matrix of a shape set, drawn on `device` with torch's
     seeded generator from the same distributions as `weight` / `grad`:
     N(0, w_std^2) weights; N(0, g_std^2), g_std * Student-t(3) (a normal over the root
     mean square of three normals), or exp(N(0,1)) row scales times N(0, g_std^2)
     gradients, rounded to bf16 when the set's gradients are bf16. Matrices whose
     index is in `exact` get the host generator's values instead, so that the oracle
-    can be run on them with identical inputs. Returns (Ws fp32, Gs) as lists."""
+    can be run on them with identical inputs. With `only` (a set of indices) just those
+    matrices are drawn, in order (a subset for profiling; its values differ from the
+    full set's). Returns (Ws fp32, Gs) as lists."""
     import torch
     gen = torch.Generator(device=device)
     gen.manual_seed(int(np.random.SeedSequence([BASE_SEED, w.wid, seed, step]).generate_state(1)[0]))
@@ -179,6 +181,8 @@ def device_inputs(w: Workload, device, seed: int = 0, exact=(), step: int = 0):
     exact = set(exact)
     Ws, Gs = [], []
     for spec in w.matrices():
+        if only is not None and spec.index not in only:
+            continue
         shape = (spec.rows, spec.cols)
         if spec.index in exact:
             Ws.append(torch.from_numpy(weight(w, spec)).to(device))

@@ -30,6 +30,15 @@ def test_roofline_names_the_dominant_tensor_kernel_and_its_fraction():
     # a timed region of a second or more is compared with the sustained figure
     r2 = bench.roofline(_prof(), w, PEAKS, "measured", "gpt160m", region_ms=1500.0)
     assert r2["peak"] == PEAKS["bf16_tflops_sustained"] and "sustained" in r2["peak_source"]
+    # so is a shorter region that ran under the power cap; both fractions are reported
+    r3 = bench.roofline(_prof(), w, PEAKS, "measured", "gpt160m", region_ms=900.0,
+                        clocks={"reasons": ["sw_power_cap"]})
+    assert r3["peak"] == PEAKS["bf16_tflops_sustained"] and "sw_power_cap" in r3["peak_source"]
+    assert r3["frac_burst"] == pytest.approx(achieved / 1600.0)
+    assert r3["frac_sustained"] == pytest.approx(achieved / 1400.0)
+    r4 = bench.roofline(_prof(), w, PEAKS, "measured", "gpt160m", region_ms=900.0,
+                        clocks={"reasons": []})
+    assert r4["peak"] == PEAKS["bf16_tflops"]
 
 
 def test_roofline_of_the_fp32_path_is_alu_bound_with_a_fraction():

@@ -16,7 +16,7 @@
 //                           64x64 tiles, one per 256-thread block, 4x4 outputs per thread.
 //   ns_simt_fused_kernel    small matrices (n <= 256): one cluster of 16 (or 8) blocks
 //                           per matrix runs all iterations and phases in a single
-//                           launch; 32x32 tiles (2x2 outputs per thread) from full-K
+//                           launch; 32x32 tiles (APPLY 32x64) from full-K
 //                           operand panels in shared memory, dealt round-robin to the
 //                           cluster's blocks, and a cluster barrier between phases, so a
 //                           step costs one launch instead of 3 per iteration.
@@ -175,14 +175,16 @@ __device__ __forceinline__ void cluster_phase_barrier() {
   cluster_sync_all();
 }
 
-// Fused kernel tile: a 32 x 32 output tile computed from full-K operand panels staged in
-// shared memory by one round of loads (K <= kFusedMaxK), so that the tile pays the L2
-// latency once instead of once per k-step. 2 x 2 outputs per thread, in k order.
-//   As[i][k] = A[i0 + i][k]                      (row stride lda_s, odd)
+// Fused kernel tile: a 32 x 32 (GRAM, POLY) or 32 x 64 (APPLY) output tile computed from
+// full-K operand panels staged in shared memory by one round of loads (K <= kFusedMaxK),
+// so that the tile pays the L2 latency once instead of once per k-step. 2 x 2 (2 x 4)
+// outputs per thread, in k order.
+//   As[i][k] = A[i0 + i][k]                      (row stride kFusedStride, odd)
 //   GRAM / POLY: Bs[j][k] = B[j0 + j][k]         (B is X, or S, which is symmetric)
-//   APPLY:       Bs[k][j] = X[k][j0 + j]          (row stride 32)
+//   APPLY:       Bs[k][j] = X[k][j0 + j]          (row stride 64)
 constexpr int kFusedMaxK = 256;
 constexpr int kFusedStride = kFusedMaxK + 1;  // odd row stride: conflict-free column reads
+constexpr int kApplyTN = 64;                  // APPLY tile columns
 
 template <int PHASE>
 __device__ __forceinline__ void fused_tile(const NsClassArgs& k, int mat, int t, const float* X,
@@ -199,7 +201,7 @@ __device__ __forceinline__ void fused_tile(const NsClassArgs& k, int mat, int t,
     while (rem >= tiles_i - ti) { rem -= tiles_i - ti; ++ti; }
     tj = ti + rem;
   } else {
-    const int tiles_j = (k.n + TT - 1) / TT;
+    const int tiles_j = (k.n + kApplyTN - 1) / kApplyTN;
     ti = t / tiles_j;
     tj = t - ti * tiles_j;
   }
@@ -211,7 +213,7 @@ __device__ __forceinline__ void fused_tile(const NsClassArgs& k, int mat, int t,
   if (PHASE == PH_GRAM) { A = X; lda = k.ldx; K = k.n; ncols = m; }
   else if (PHASE == PH_POLY) { A = S; lda = k.lds; K = m; ncols = m; }
   else { A = Pm; lda = k.lds; K = m; ncols = k.n; }
-  const int i0 = ti * TT, j0 = tj * TT;
+  const int i0 = ti * TT, j0 = tj * (PHASE == PH_APPLY ? kApplyTN : TT);
   // panels: every load of the tile is issued before any shared-memory store (16-byte
   // loads; warp w takes rows w, w + 8, w + 16, w + 24, lanes along k). Rows start on
   // 256-byte boundaries (slab leading dimensions are multiples of 64); values past K
@@ -251,35 +253,44 @@ __device__ __forceinline__ void fused_tile(const NsClassArgs& k, int mat, int t,
       }
     }
   }
-  if (PHASE == PH_APPLY) {  // Bs[k][j] = X[k][j0 + j]: K rows of 32, 8 loads in flight
-    const int gj = j0 + lane;
+  if (PHASE == PH_APPLY) {  // Bs[k][j] = X[k][j0 + j]: K rows of 64, 8 loads in flight
+    const int gj = j0 + 2 * lane;  // two columns per lane (8-byte loads; ldx and j0 are even)
     for (int kb = warp; kb < K; kb += 8 * (NT / 32)) {
-      float v[8];
+      float2 v[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int kk = kb + q * (NT / 32);
-        v[q] = (kk < K && gj < ncols) ? X[(int64_t)kk * k.ldx + gj] : 0.f;
+        const float* src = X + (int64_t)kk * k.ldx + gj;
+        v[q] = make_float2(0.f, 0.f);
+        if (kk < K && gj + 1 < ncols) v[q] = *reinterpret_cast<const float2*>(src);
+        else if (kk < K && gj < ncols) v[q].x = src[0];
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int kk = kb + q * (NT / 32);
-        if (kk < K) Bs[kk * TT + lane] = v[q];
+        if (kk < K) *reinterpret_cast<float2*>(Bs + kk * kApplyTN + 2 * lane) = v[q];
       }
     }
   }
   __syncthreads();
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  constexpr int NY = PHASE == PH_APPLY ? 4 : 2;  // output columns per thread
+  float acc[2][NY];
+#pragma unroll
+  for (int x = 0; x < 2; ++x)
+#pragma unroll
+    for (int y = 0; y < NY; ++y) acc[x][y] = 0.f;
   const float* a0 = As + (ty * 2) * kFusedStride;
   const float* a1 = a0 + kFusedStride;
   if (PHASE == PH_APPLY) {
     for (int kk = 0; kk < K; ++kk) {
-      const float av0 = a0[kk], av1 = a1[kk];
-      const float2 bv = *reinterpret_cast<const float2*>(Bs + kk * TT + tx * 2);
-      acc[0][0] = fmaf(av0, bv.x, acc[0][0]);
-      acc[0][1] = fmaf(av0, bv.y, acc[0][1]);
-      acc[1][0] = fmaf(av1, bv.x, acc[1][0]);
-      acc[1][1] = fmaf(av1, bv.y, acc[1][1]);
+      const float av[2] = {a0[kk], a1[kk]};
+      const float4 bq = *reinterpret_cast<const float4*>(Bs + kk * kApplyTN + tx * 4);
+      const float bv[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < NY; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
     }
   } else {
     const float* b0 = Bs + (tx * 2) * kFusedStride;
@@ -297,8 +308,8 @@ __device__ __forceinline__ void fused_tile(const NsClassArgs& k, int mat, int t,
     const int i = i0 + ty * 2 + x;
     if (i >= m) continue;
 #pragma unroll
-    for (int y = 0; y < 2; ++y) {
-      const int j = j0 + tx * 2 + y;
+    for (int y = 0; y < NY; ++y) {
+      const int j = j0 + tx * NY + y;
       if (j >= ncols) continue;
       if (PHASE == PH_GRAM) {
         const float v = scale * acc[x][y];
@@ -328,8 +339,9 @@ __global__ void __launch_bounds__(NT) ns_simt_fused_kernel(const NsFusedArgs a) 
   while (c + 1 < a.num_classes && gm >= a.mat_base[c + 1]) ++c;
   const NsClassArgs& k = a.cls[c];
   const int mat = gm - a.mat_base[c];
-  const int ti = (k.m + 31) / 32, tj = (k.n + 31) / 32;
-  const int sym_tiles = ti * (ti + 1) / 2, apply_tiles = ti * tj;
+  const int ti = (k.m + 31) / 32;
+  const int sym_tiles = ti * (ti + 1) / 2;
+  const int apply_tiles = ti * ((k.n + kApplyTN - 1) / kApplyTN);
   for (int it = 0; it < a.steps; ++it) {
     const float* x_in = static_cast<const float*>((it & 1) ? a.x1[c] : a.x0[c]) + mat * k.xstride;
     float* x_out = static_cast<float*>((it & 1) ? a.x0[c] : a.x1[c]) + mat * k.xstride;
@@ -348,10 +360,11 @@ __global__ void __launch_bounds__(NT) ns_simt_fused_kernel(const NsFusedArgs a) 
   }
 }
 
-// As (32 rows) and the larger of the two B layouts: 32 rows of K, or K rows of 32
+// As (32 rows) and the larger of the two B layouts: 32 rows of K, or K rows of 64
 constexpr size_t kFusedSmem =
-    sizeof(float) * (32 * kFusedStride +
-                     (32 * kFusedStride > kFusedMaxK * 32 ? 32 * kFusedStride : kFusedMaxK * 32));
+    sizeof(float) * (32 * kFusedStride + (32 * kFusedStride > kFusedMaxK * kApplyTN
+                                              ? 32 * kFusedStride
+                                              : kFusedMaxK * kApplyTN));
 
 }  // namespace
 

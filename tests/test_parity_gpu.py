@@ -394,3 +394,35 @@ def test_plan_graph_replay_matches_eager_steps(env):
         assert H.rel(runs[0][1][i], runs[1][1][i]) <= 1e-6, i
         for key in ("w_norm", "o_norm"):
             assert abs(runs[0][2][i][key] - runs[1][2][i][key]) <= 1e-5 * abs(runs[1][2][i][key]) + 1e-9
+
+
+def test_fp32_fused_and_per_phase_classes_in_one_plan(env):
+    """The fp32 path with six shape classes in one plan (classes are keyed by the oriented
+    (m, n), so 64x200 and 200x64 share one): five small ones (n <= 256) run all iterations
+    in the fused cluster kernel, in two launches of at most four classes; the 300x520 class
+    takes one launch per phase. 10 steps, 1e-4 against the oracle."""
+    B, torch = env
+    shapes = [(9, 13), (64, 200), (256, 100), (128, 256), (200, 64), (300, 520), (520, 300),
+              (1, 256)]
+    W0 = [H.seeded(r, c, 1900 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded(r, c, 2000 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(10)]
+    hp = H.gpu_hp(B, mode="muongs", wd=0.1, ns_fp32=True)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.float32)
+    worst = H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs", wd=0.1), H.TOL_FP32)
+    print(f"\nFP32 MIXED: max rel err W {worst['W']:.2e} M {worst['M']:.2e} dW {worst['dW']:.2e}")
+
+
+@pytest.mark.parametrize("m", [64, 130, 192, 320, 448, 500, 640])
+def test_single_cta_variable_width_tiles_ragged_m(env, m):
+    """Single-CTA classes (m not a multiple of 256) cut every 128-row block of S and P'
+    into variable-width column pieces; m values whose row blocks end ragged, whose pieces
+    are 64, 128, 192 or 256 wide, and whose B units switch from K-major to mirrored inside
+    a piece. 16 matrices per class (the piece order rotates per matrix), 3 steps."""
+    B, torch = env
+    shapes = [(m, m + 192)] * 8 + [(m + 320, m)] * 8
+    W0 = [H.seeded(r, c, 2100 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded_bf16(r, c, 2200 + 20 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(3)]
+    gpu = H.run_steps(B, torch, W0, grads, H.gpu_hp(B, mode="muongs"), torch.bfloat16)
+    H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs"), H.TOL_BF16)

@@ -62,6 +62,7 @@ constexpr int BM = 128, BK = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kThreadsTc = 64 + 32 * kEpiWarps;  // 320
 constexpr int kWarpBoxBytes = 32 * 128;           // one 32-row x 64-column bf16 output box
+constexpr int kMaxStages = 8;                     // barrier pairs reserved for the operand ring
 
 template <int BN, int PHASE, bool PAIR>
 struct TcCfg {
@@ -82,15 +83,22 @@ struct TcCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   // epilogue: each warp stores 32 x 64 boxes; it takes every other 64-column chunk
   static constexpr int kChunksPerWarp = kNCol / 128;
-  static constexpr int kEpiBufs = (PAIR && kChunksPerWarp >= 2) ? 2 : 1;  // per-warp box buffers
+  // one box buffer per warp: the epilogue has slack (it waits for the accumulator most of
+  // the time), and the shared memory goes to the operand ring instead
+  static constexpr int kEpiBufs = 1;
   static constexpr int kStagingBytes =
       kCStaged ? BM * kNCol * 2 : kEpiWarps * kEpiBufs * kWarpBoxBytes;  // C tile, or per-warp boxes
   static constexpr int kBudget = 224 * 1024;
   static constexpr int kFit = (kBudget - kStagingBytes) / kStageBytes;
-  static constexpr int kStages = kFit > 8 ? 8 : kFit;
+  static constexpr int kStages = kFit > kMaxStages ? kMaxStages : kFit;
   static constexpr int kOffStg = kStages * kStageBytes;
   static constexpr int kOffBar = kOffStg + kStagingBytes;
+  static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kTmemCols = 2 * kNCol;
+  // barrier region: full and empty per ring slot, tfull and tempty per accumulator, done,
+  // cfull, the TMEM address, the abort flag and one stage_meta word per ring slot
+  static_assert(8 * (2 * kMaxStages + 2 + 2 + 2) + 4 + 4 + 4 * kMaxStages <= 256,
+                "barrier region overflow");
   static constexpr int kSmemBytes = kOffBar + 256 + 1024;
   static constexpr int kMmaM = PAIR ? 256 : 128;
   static constexpr int kMmaN = PAIR ? 256 : BN;
@@ -152,10 +160,54 @@ __device__ __forceinline__ TileJob decode(const NsPhaseArgs& p, int t, bool sym,
   return j;
 }
 
+// The class of tile t (the first part of decode, for roles that need no more).
+__device__ __forceinline__ int class_of(const NsPhaseArgs& p, int t) {
+  int c = 0;
+  while (c + 1 < p.num_classes && t >= p.tile_base[c + 1]) ++c;
+  return c;
+}
+
+// Stage descriptor of a variable-width tile, written by the producer for the MMA issuer
+// (which then decodes nothing): B's unit count, the first mirrored unit, A's layout, and
+// whether A is B's first rows.
+__device__ __forceinline__ uint32_t stage_meta(int nu, int split, bool a_t, bool shared_a) {
+  return static_cast<uint32_t>(nu) | (static_cast<uint32_t>(split) << 3) |
+         (a_t ? (1u << 6) : 0u) | (shared_a ? (1u << 7) : 0u);
+}
+
 // Whether B unit u (64 rows starting at output column col0 + 64 u) of k-block kb lies
 // below the stored 128-block diagonal (variable-width symmetric tiles).
 __device__ __forceinline__ bool unit_mirrored(bool sym_operand, int col0, int u, int kb) {
   return sym_operand && (kb * 64) / 128 < (col0 + 64 * u) / 128;
+}
+
+// Whether a tile's A operand is already in shared memory as the start of its B operand.
+// In GRAM (A = B = X) and POLY (A = B = S) a tile on the block diagonal reads the same
+// rows for both operands, with the same layout decision in every k-block (below_diag and
+// unit_mirrored agree when the tile's first column is its first row): the tile then loads
+// only B, and the MMA takes A from B's first 128 rows. A single-CTA piece needs at least
+// two B units (128 rows); a CTA of a pair owns 128 rows of each.
+__device__ __forceinline__ bool a_in_b(bool sym, bool varn, const TileJob& j, int tile_m) {
+  if (!sym) return false;
+  return varn ? (j.col0 == j.ti * tile_m && j.nt >= 128) : j.ti == j.tj;
+}
+
+// Stage size of a launch of variable-width symmetric tiles: the largest k-block of A and
+// B that any of its tiles loads (B alone where a_in_b). The ring of fixed size then holds
+// as many stages as fit (narrow pieces and diagonal tiles leave room for more).
+__device__ __forceinline__ int varn_stage_bytes(const NsPhaseArgs& p, int a_bytes) {
+  int most = 0;
+  for (int c = 0; c < p.num_classes; ++c) {
+    const int m = p.cls[c].m;
+    for (int i = 0; i < sym_row_blocks(m); ++i)
+      for (int jj = 0; jj < sym_pieces(m, i); ++jj) {
+        int col0, width;
+        sym_piece(m, i, jj, &col0, &width);
+        const int bytes = (col0 == 128 * i && width >= 128 ? 0 : a_bytes) + width * (BK * 2);
+        most = bytes > most ? bytes : most;
+      }
+  }
+  return most;
 }
 
 // Byte offset of element (r, c) of a 128-row tile staged as 64-column boxes with
@@ -196,7 +248,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
   constexpr bool SYM = C::kSym;
   constexpr bool HAS_C = C::kCStaged;        // C tile staged in shared memory by TMA
   constexpr bool C_REGS = C::kCRegs;         // C read into registers from global memory
-  constexpr int S = C::kStages;
   constexpr bool A_SYM = PHASE != PH_GRAM;   // A is S (POLY) or P' (APPLY): upper blocks only
   constexpr bool B_SYM = PHASE == PH_POLY;   // B is S
   constexpr bool B_MN = PHASE == PH_APPLY;   // B is X read along its rows
@@ -207,16 +258,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* stg = smem + C::kOffStg;  // output staging (POLY: the C tile, overwritten by D)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* empty = full + S;
-  uint64_t* tfull = empty + S;
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* tfull = empty + kMaxStages;
   uint64_t* tempty = tfull + 2;
   uint64_t* done = tempty + 2;
   uint64_t* cfull = done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(cfull + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* meta = tmem_slot + 2;  // per ring slot: stage_meta (variable-width tiles)
 
   const NsPhaseArgs& p = P.args;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // operand ring: S stages of sbytes (variable-width tiles size them to the launch)
+  int sbytes = C::kStageBytes;
+  if (VARN) {
+    sbytes = varn_stage_bytes(p, C::kABytes);
+    sbytes = sbytes < 1024 ? 1024 : sbytes;
+  }
+  const int S_ = C::kRingBytes / sbytes;
+  const int S = S_ > kMaxStages ? kMaxStages : S_;
   const int total = p.tile_base[p.num_classes];
   const int rank = PAIR ? static_cast<int>(cluster_cta_rank()) : 0;
   const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
@@ -261,7 +321,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
         tma_prefetch(&P.ta[c]);
         tma_prefetch(&P.tb[c]);
       }
-      long long q = 0;
+      long long q = 0;        // stages loaded
+      int s = 0;              // its slot, q mod S
+      uint32_t par = 0;       // and the parity of the slot's use, (q / S) mod 2
       bool ok = true;
       for (int t = unit; t < total && ok; t += nunits) {
         const TileJob j = decode(p, t, SYM, VARN, C::kTileN);
@@ -269,34 +331,52 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
         const int a_row0 = j.ti * C::kTileM + rank * 128;
         const int b_row0 = j.col0 + rank * (PAIR ? 128 : 0);
         for (int kb = 0; kb < kb_n; ++kb) {
-          const int s = static_cast<int>(q % S);
-          const uint32_t par = static_cast<uint32_t>((q / S) & 1);
           if (!mbar_wait(&empty[s], par ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + s * C::kStageBytes;
+          uint8_t* sa = smem + s * sbytes;
           uint8_t* sb = sa + C::kABytes;
           if (VARN) {
             // A: the row block's 128 rows; B: the tile's nt rows in 64-row units, each
-            // K-major (a 64 x 64 box) or, below the diagonal, its mirror (one chunk)
-            mbar_expect_tx(&full[s], C::kABytes + j.nt * (BK * 2));
-            load_k_block<false>(sa, &P.ta[j.c], &P.ta_t[j.c], &full[s], a_row0, kb, j.mat,
-                                below_diag(A_SYM, j.ti * C::kTileM, kb, C::kTileM));
-            for (int u = 0; u < j.nt / 64; ++u) {
+            // K-major (a 64 x 64 box) or, below the diagonal, its mirror (one chunk).
+            // Without an A of its own the stage starts with B.
+            const bool shared_a = a_in_b(SYM, true, j, C::kTileM);
+            const bool a_t = below_diag(A_SYM, j.ti * C::kTileM, kb, C::kTileM);
+            const int nu = j.nt / 64;
+            int split = nu;  // first mirrored unit (unit_mirrored is monotone in u)
+            for (int u = 0; u < nu; ++u)
+              if (unit_mirrored(B_SYM, j.col0, u, kb)) { split = u; break; }
+            // published to the MMA issuer by the arrive below (release, CTA scope)
+            meta[s] = stage_meta(nu, split, a_t, shared_a);
+            if (shared_a) sb = sa;
+            mbar_expect_tx(&full[s], (shared_a ? 0 : C::kABytes) + j.nt * (BK * 2));
+            if (!shared_a)
+              load_k_block<false>(sa, &P.ta[j.c], &P.ta_t[j.c], &full[s], a_row0, kb, j.mat, a_t);
+            // Two neighbouring units of the same layout come in one 128-row box through
+            // A's maps (A and B are the same slab in GRAM and POLY): fewer, larger copies
+            for (int u = 0; u < nu;) {
               uint8_t* dst = sb + u * (64 * BK * 2);
-              if (unit_mirrored(B_SYM, j.col0, u, kb))
-                tma_load_4d(dst, &P.tb_t[j.c], &full[s], 0, kb * BK, j.col0 / 64 + u, j.mat);
-              else
-                tma_load_3d(dst, &P.tb[j.c], &full[s], kb * BK, j.col0 + 64 * u, j.mat);
+              const bool mir = u >= split;
+              const bool two = u + 1 < nu && (u + 1 >= split) == mir;
+              const CUtensorMap* km = two ? &P.ta[j.c] : &P.tb[j.c];
+              const CUtensorMap* mm = two ? &P.ta_t[j.c] : &P.tb_t[j.c];
+              if (mir) tma_load_4d(dst, mm, &full[s], 0, kb * BK, j.col0 / 64 + u, j.mat);
+              else tma_load_3d(dst, km, &full[s], kb * BK, j.col0 + 64 * u, j.mat);
+              u += two ? 2 : 1;
             }
             ++q;
+            if (++s == S) s = 0, par ^= 1u;
             continue;
           }
-          if (!PAIR || rank == 0) mbar_expect_tx(&full[s], (PAIR ? 2 : 1) * C::kStageBytes);
+          const bool shared_a = a_in_b(SYM, false, j, C::kTileM);
+          if (!PAIR || rank == 0)
+            mbar_expect_tx(&full[s], (PAIR ? 2 : 1) * (shared_a ? C::kABytes : C::kStageBytes));
           load_k_block<PAIR>(sa, &P.ta[j.c], &P.ta_t[j.c], &full[s], a_row0, kb, j.mat,
                              below_diag(A_SYM, j.ti * C::kTileM, kb, C::kTileM));
-          if (!B_MN) {
+          if (shared_a) {
+            // diagonal tile: B's rows are A's (the MMA reads both from the A stage)
+          } else if (!B_MN) {
             load_k_block<PAIR>(sb, &P.tb[j.c], &P.tb_t[j.c], &full[s], b_row0, kb, j.mat,
                                below_diag(B_SYM, j.tj * C::kTileN, kb, C::kTileN));
           } else {  // X rows kb*BK.., columns b_row0.. in kBRows/64 chunks, one box
@@ -304,6 +384,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
             else tma_load_4d(sb, &P.tb[j.c], &full[s], 0, kb * BK, b_row0 / 64, j.mat);
           }
           ++q;
+          if (++s == S) s = 0, par ^= 1u;
         }
       }
       if (!ok) {
@@ -314,7 +395,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
       // first CTA's full barriers count both CTAs' bytes).
       if (!PAIR || rank == 0)
         for (long long r = (q > S ? q - S : 0); r < q; ++r)
-          mbar_wait(&full[r % S], static_cast<uint32_t>((r / S) & 1), nullptr);
+          mbar_wait(&full[static_cast<int>(r % S)], static_cast<uint32_t>((r / S) & 1), nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -325,11 +406,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
       // chunks; both SBO 1024 B) and add the address per slice
       const uint64_t kmaj_hi = smem_desc_sw128(0, 16, 1024);
       const uint64_t mnmaj_hi = smem_desc_sw128(0, 64 * BK * 2, 1024);
-      long long q = 0;
+      int s = 0;              // slot of the next stage
+      uint32_t par = 0;       // parity of that slot's use
       int it = 0;
       bool ok = true;
       for (int t = unit; t < total && ok; t += nunits, ++it) {
-        const TileJob j = decode(p, t, SYM, VARN, C::kTileN);
+        // variable-width tiles: the producer describes each stage (meta); other tiles
+        // are decoded here
+        const TileJob j = VARN ? TileJob{class_of(p, t), 0, 0, 0, 0, 0}
+                               : decode(p, t, SYM, VARN, C::kTileN);
         const int kb_n = p.cls[j.c].k_blocks;
         const int a_row0 = j.ti * C::kTileM;  // the first CTA's rows decide for both
         const int b_row0 = j.col0;
@@ -342,8 +427,6 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(ab * C::kNCol);
         for (int kb = 0; kb < kb_n; ++kb) {
-          const int s = static_cast<int>(q % S);
-          const uint32_t par = static_cast<uint32_t>((q / S) & 1);
           if (!mbar_wait(&full[s], par, abort_flag)) {
             ok = false;
             break;
@@ -353,15 +436,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
             // B's 64-row units switch from K-major to mirrored (MN-major) at most once
             // along the tile (unit_mirrored is monotone in u): one MMA per run of units
             // of the same layout, each writing its own accumulator columns
-            const bool a_t = below_diag(A_SYM, a_row0, kb, C::kTileM);
-            const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
-            const uint32_t sb = sa + C::kABytes;
+            const uint32_t md = meta[s];
+            const int nu = static_cast<int>(md & 7u), split = static_cast<int>((md >> 3) & 7u);
+            const bool a_t = (md >> 6) & 1u, shared_a = (md >> 7) & 1u;
+            const uint32_t sa = smem_u32(smem + s * sbytes);
+            const uint32_t sb = shared_a ? sa : sa + C::kABytes;
             const uint64_t ad0 = (a_t ? mnmaj_hi : kmaj_hi) | static_cast<uint64_t>((sa >> 4) & 0x3FFFu);
             const uint64_t astep = a_t ? 128u : 2u;
-            const int nu = j.nt / 64;
-            int split = nu;  // first mirrored unit
-            for (int u = 0; u < nu; ++u)
-              if (unit_mirrored(B_SYM, j.col0, u, kb)) { split = u; break; }
 #pragma unroll
             for (int run = 0; run < 2; ++run) {
               const int u0 = run == 0 ? 0 : split, u1 = run == 0 ? split : nu;
@@ -378,7 +459,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
                          idesc, (kb | kk) != 0 ? 1u : 0u);
             }
             umma_commit(&empty[s]);
-            ++q;
+            if (++s == S) s = 0, par ^= 1u;
             continue;
           }
           // one instruction serves both CTAs of a pair: the layout choice is made per
@@ -386,8 +467,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           const bool a_t = below_diag(A_SYM, a_row0, kb, C::kTileM);
           const bool b_t = B_MN || below_diag(B_SYM, b_row0, kb, C::kTileN);
           const uint32_t idesc = idesc0 | (a_t ? (1u << 15) : 0u) | (b_t ? (1u << 16) : 0u);
-          const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
-          const uint32_t sb = sa + C::kABytes;
+          const uint32_t sa = smem_u32(smem + s * sbytes);
+          const uint32_t sb = a_in_b(SYM, false, j, C::kTileM) ? sa : sa + C::kABytes;
           // K-major slices advance 32 B (2 in the >>4 address field), MN-major 2 KB (128)
           const uint64_t ad0 = (a_t ? mnmaj_hi : kmaj_hi) | static_cast<uint64_t>((sa >> 4) & 0x3FFFu);
           const uint64_t bd0 = (b_t ? mnmaj_hi : kmaj_hi) | static_cast<uint64_t>((sb >> 4) & 0x3FFFu);
@@ -405,7 +486,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) ns_tc_kernel(const __grid_const
           } else {
             umma_commit(&empty[s]);
           }
-          ++q;
+          if (++s == S) s = 0, par ^= 1u;
         }
         if (!ok) break;
         if (PAIR) {

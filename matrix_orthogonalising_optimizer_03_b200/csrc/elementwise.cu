@@ -15,10 +15,14 @@
 // per thread, 128-bit accesses when aligned; the reductions and post_apply take two
 // 32-row sub-tiles at a time, all their loads issued before any arithmetic). The
 // super-tile of each block is found by binary search over a per-matrix tile prefix.
+// Without equilibration and with aligned rows, the reduction instead stages its loads in
+// shared memory with cp.async (post_reduce_staged_kernel).
 // Per-matrix sums use one atomic per block; the equilibration row / column sums are
 // reduced inside the block (shuffles, and shared memory across warps for columns) and
 // use one atomic per row and per column of the super-tile.
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "muon_internal.h"
 #include "elementwise.h"
@@ -450,6 +454,147 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
   }
 }
 
+// ------------------------------------------------------------------ post_reduce (staged)
+// The three per-matrix sums with the loads moved out of the registers: every thread copies its
+// share of each 32 x 64 sub-tile (W rows and slab rows, 16 bytes per copy) into a ring of
+// shared-memory stages with cp.async, kStg - 1 sub-tiles ahead of the arithmetic, and
+// reads its 8 elements back from shared memory. Bytes in flight per SM are then set by
+// the ring (4 blocks x 4 stages of 12 KB), not by the registers that hold pending
+// loads. Used when every W row segment of the plan is 16-byte aligned (rows of 16-byte
+// multiples, 4 | cols), the slab is bf16 and the step has no equilibration (with the
+// per-row and per-column sums as well, the register-staged kernel above measured
+// faster). For tall matrices a stage holds 64 slab rows of 64 bytes (32 storage rows of
+// one storage column each), skewed by 16 bytes every 8 rows so that the column reads
+// below meet no bank conflict.
+constexpr int kStg = 4;                              // ring stages
+constexpr int kStgW = kTR * kTC * 4;                 // W sub-tile, rows at 256 bytes
+constexpr int kStgO = kTC * kTR * 2 + 8 * 16;        // O sub-tile (tall: skewed rows)
+constexpr int kStgBytes = kStgW + kStgO;
+constexpr int kStgSmem = kStg * kStgBytes + 128;     // dynamic shared memory (+ alignment)
+static_assert(kStgBytes % 128 == 0, "stage alignment");
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Byte offset, in a stage's O part, of slab row k of a tall sub-tile.
+__device__ __forceinline__ int o_tall_off(int k) { return k * 64 + (k >> 3) * 16; }
+
+// This thread's copies of sub-tile (r0, c0) of matrix d into stage st: two 16-byte pieces
+// of W (512 per sub-tile) and one of the slab (256). Pieces outside the matrix are not
+// copied (the arithmetic masks them).
+__device__ __forceinline__ void stage_subtile(const DevMat& d, const DevSlab& s, bool tall, int r0,
+                                              int c0, uint8_t* st) {
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int q = tid + h * kThreads, row = q >> 4, col = (q & 15) * 4;
+    if (r0 + row < d.rows && c0 + col < d.cols)
+      cp_async16(st + row * (kTC * 4) + col * 4, d.W + static_cast<int64_t>(r0 + row) * d.ld_w + c0 + col);
+  }
+  const uint16_t* slab = static_cast<const uint16_t*>(s.xf);
+  if (!tall) {
+    const int row = tid >> 3, col = (tid & 7) * 8;
+    if (r0 + row < d.rows)
+      cp_async16(st + kStgW + row * (kTC * 2) + col * 2, slab + static_cast<int64_t>(r0 + row) * s.ldx + c0 + col);
+  } else {
+    const int k = tid >> 2, col = (tid & 3) * 8;  // slab row c0 + k, slab columns r0 + col ..
+    if (c0 + k < d.cols)
+      cp_async16(st + kStgW + o_tall_off(k) + col * 2, slab + static_cast<int64_t>(c0 + k) * s.ldx + r0 + col);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 4) post_reduce_staged_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) &
+                                             ~static_cast<uintptr_t>(127));
+  __shared__ double red[3][kThreads / 32];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int sub_r = a.sub_r, sub_c = a.sub_c;
+  const int tiles_c = (d.cols + sub_c * kTC - 1) / (sub_c * kTC);
+  const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  // sub-tiles of the super-tile inside the matrix, band by band (64 columns each)
+  const int nbr = min(sub_r, (d.rows - R0 + kTR - 1) / kTR);
+  const int nbc = min(sub_c, (d.cols - C0 + kTC - 1) / kTC);
+  const int nsub = nbr * nbc;
+  // the first kStg - 1 stages in flight (one commit group per stage, empty ones too)
+#pragma unroll
+  for (int i = 0; i < kStg - 1; ++i) {
+    if (i < nsub) stage_subtile(d, s, tall, R0 + (i % nbr) * kTR, C0 + (i / nbr) * kTC, ring + i * kStgBytes);
+    cp_async_commit();
+  }
+
+  float ww = 0.f, wo = 0.f, oo = 0.f;
+  for (int i = 0; i < nsub; ++i) {
+    const int slot = i % kStg, g = i % nbr, bj = i / nbr;  // band-major order
+    const int r0 = R0 + g * kTR, c0 = C0 + bj * kTC;
+    const uint8_t* st = ring + slot * kStgBytes;
+    {  // stage i + kStg - 1 goes into the slot freed at the end of the previous iteration
+      const int in = i + kStg - 1;
+      if (in < nsub)
+        stage_subtile(d, s, tall, R0 + (in % nbr) * kTR, C0 + (in / nbr) * kTC, ring + (in % kStg) * kStgBytes);
+      cp_async_commit();
+    }
+    cp_async_wait<kStg - 1>();  // this thread's copies of stage i have landed
+    __syncthreads();            // and everyone's
+    const int r = r0 + lr, c = c0 + lc;
+    const int valid = r < d.rows ? max(0, min(8, d.cols - c)) : 0;
+    float w[8], o[8];
+    {
+      const float4 x = *reinterpret_cast<const float4*>(st + lr * (kTC * 4) + lc * 4);
+      const float4 y = *reinterpret_cast<const float4*>(st + lr * (kTC * 4) + lc * 4 + 16);
+      w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+      w[4] = y.x; w[5] = y.y; w[6] = y.z; w[7] = y.w;
+    }
+    if (!tall) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(st + kStgW + lr * (kTC * 2) + lc * 2);
+      const uint32_t q[4] = {ov.x, ov.y, ov.z, ov.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        o[2 * e] = __uint_as_float(q[e] << 16);
+        o[2 * e + 1] = __uint_as_float(q[e] & 0xFFFF0000u);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        o[e] = __uint_as_float(static_cast<uint32_t>(
+                   *reinterpret_cast<const uint16_t*>(st + kStgW + o_tall_off(lc + e) + lr * 2))
+               << 16);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {  // stale shared memory outside the matrix counts as 0
+      const float we = e < valid ? w[e] : 0.f, oe = e < valid ? o[e] : 0.f;
+      const float o2 = oe * oe, wov = we * oe;
+      ww = fmaf(we, we, ww);
+      wo += wov;
+      oo += o2;
+    }
+    // every thread is done with this stage before it is refilled
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+  double acc[3] = {ww, wo, oo};
+  block_sum<3>(acc, red);
+  if (threadIdx.x == 0) {
+    atomicAdd(&a.scal[k].w2, acc[0]);
+    atomicAdd(&a.scal[k].wo, acc[1]);
+    atomicAdd(&a.scal[k].o2, acc[2]);
+  }
+}
+
 // ------------------------------------------------------------------ post_finalize
 __device__ __forceinline__ double block_sum2(double& x, double& y, double (*sh)[kThreads / 32]) {
   double v[2] = {x, y};
@@ -698,8 +843,36 @@ cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
   ingest_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
+// Staged reduction: needs more than the default 48 KB of dynamic shared memory; the
+// opt-in is a per-device attribute, set once on each device.
+cudaError_t launch_reduce_staged(const ElemArgs& a, cudaStream_t s) {
+  static std::atomic<uint64_t> attr_devices{0};
+  auto kern = post_reduce_staged_kernel;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
+  if (bit == 0 || !(attr_devices.load(std::memory_order_acquire) & bit)) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStgSmem);
+    if (e != cudaSuccess) return e;
+    attr_devices.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.total_tiles, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kStgSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
+  if (a.staged && !a.x_fp32 && !a.equilibrate) return launch_reduce_staged(a, s);
   if (a.equilibrate)
     return a.x_fp32 ? launch_pdl(post_reduce_eq_kernel<true>, a.total_tiles, s, a)
                     : launch_pdl(post_reduce_eq_kernel<false>, a.total_tiles, s, a);

@@ -65,6 +65,7 @@ struct muon_plan_s {
   std::vector<int32_t> tile_prefix;
   int64_t eq_total = 0;
   int sub_r = 4, sub_c = 4;  // elementwise super-tile in 32 x 64 sub-tiles
+  bool staged = false;       // staged (shared-memory ring) post_reduce
   size_t off_scal = 0, off_coef = 0, off_desc = 0, off_slabs = 0, off_tiles = 0;
   size_t off_eq_o2 = 0, off_eq_wo = 0, ws_bytes = 0;
   // cached per workspace pointer and device
@@ -261,6 +262,12 @@ void build_plan(muon_plan_s* p) {
   p->sub_r = elems <= kElemSmallStep ? 1 : kElemTileR / kElemSubR;
   p->sub_c = elems <= kElemSmallStep ? 1 : kElemTileC / kElemSubC;
   const int tr = p->sub_r * kElemSubR, tc = p->sub_c * kElemSubC;
+  // the staged (plain) reduction copies W rows and slab rows in 16-byte pieces with
+  // cp.async: 16-byte aligned rows of 16-byte multiples; worth it only with several
+  // sub-tiles per block
+  p->staged = !p->x_fp32 && p->sub_r * p->sub_c > 1;
+  for (int i = 0; i < n; ++i)
+    p->staged = p->staged && (p->dev[i].flags & MAT_VEC_OK) != 0 && p->dev[i].cols % 4 == 0;
   p->tile_prefix.assign(n + 1, 0);
   for (int i = 0; i < n; ++i) {
     const int64_t t = int64_t((p->dev[i].rows + tr - 1) / tr) * ((p->dev[i].cols + tc - 1) / tc);
@@ -586,6 +593,7 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
   ea.xs_from_u2 = p->ns_steps == 0 ? 1 : 0;
   ea.sub_r = p->sub_r;
   ea.sub_c = p->sub_c;
+  ea.staged = p->staged ? 1 : 0;
 
   {
     ProfScope ps(p, stream);

@@ -819,6 +819,84 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs 
   }
 }
 
+// post_apply with the W and slab loads staged in shared memory (cp.async, the ring of
+// post_reduce_staged_kernel); the updated W goes straight from the registers to memory.
+__global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) &
+                                             ~static_cast<uintptr_t>(127));
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int sub_r = a.sub_r, sub_c = a.sub_c;
+  const int tiles_c = (d.cols + sub_c * kTC - 1) / (sub_c * kTC);
+  const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  const MatCoef cf = a.coef[k];
+  const int nbr = min(sub_r, (d.rows - R0 + kTR - 1) / kTR);
+  const int nbc = min(sub_c, (d.cols - C0 + kTC - 1) / kTC);
+  const int nsub = nbr * nbc;
+#pragma unroll
+  for (int i = 0; i < kStg - 1; ++i) {
+    if (i < nsub) stage_subtile(d, s, tall, R0 + (i % nbr) * kTR, C0 + (i / nbr) * kTC, ring + i * kStgBytes);
+    cp_async_commit();
+  }
+  for (int i = 0; i < nsub; ++i) {
+    const int slot = i % kStg;
+    const int r0 = R0 + (i % nbr) * kTR, c0 = C0 + (i / nbr) * kTC;
+    const uint8_t* st = ring + slot * kStgBytes;
+    {
+      const int in = i + kStg - 1;
+      if (in < nsub)
+        stage_subtile(d, s, tall, R0 + (in % nbr) * kTR, C0 + (in / nbr) * kTC, ring + (in % kStg) * kStgBytes);
+      cp_async_commit();
+    }
+    cp_async_wait<kStg - 1>();
+    __syncthreads();
+    const int r = r0 + lr, c = c0 + lc;
+    const int valid = r < d.rows ? max(0, min(8, d.cols - c)) : 0;
+    if (valid > 0) {
+      float w[8], o[8];
+      {
+        const float4 x = *reinterpret_cast<const float4*>(st + lr * (kTC * 4) + lc * 4);
+        const float4 y = *reinterpret_cast<const float4*>(st + lr * (kTC * 4) + lc * 4 + 16);
+        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+        w[4] = y.x; w[5] = y.y; w[6] = y.z; w[7] = y.w;
+      }
+      if (!tall) {
+        const uint4 ov = *reinterpret_cast<const uint4*>(st + kStgW + lr * (kTC * 2) + lc * 2);
+        const uint32_t q[4] = {ov.x, ov.y, ov.z, ov.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          o[2 * e] = __uint_as_float(q[e] << 16);
+          o[2 * e + 1] = __uint_as_float(q[e] & 0xFFFF0000u);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          o[e] = __uint_as_float(static_cast<uint32_t>(
+                     *reinterpret_cast<const uint16_t*>(st + kStgW + o_tall_off(lc + e) + lr * 2))
+                 << 16);
+      }
+      const float rowf = (cf.axis & 1) ? a.eq_o2[s.eq_off + r] : 1.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float f = rowf;
+        if ((cf.axis & 2) && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+        w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
+      }
+      store8_f32(d.W + static_cast<int64_t>(r) * d.ld_w + c, true, valid, w);
+    }
+    __syncthreads();  // every thread is done with this stage before it is refilled
+  }
+  cp_async_wait<0>();
+}
+
 }  // namespace
 
 // Launch with programmatic stream serialisation: the kernel may start while its
@@ -843,11 +921,11 @@ cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
   ingest_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
   return cudaGetLastError();
 }
-// Staged reduction: needs more than the default 48 KB of dynamic shared memory; the
-// opt-in is a per-device attribute, set once on each device.
-cudaError_t launch_reduce_staged(const ElemArgs& a, cudaStream_t s) {
+// Shared-memory staged kernels: they need more than the default 48 KB of dynamic shared
+// memory; the opt-in is a per-device attribute, set once on each device (per kernel).
+template <void (*kern)(ElemArgs)>
+cudaError_t launch_staged_impl(const ElemArgs& a, cudaStream_t s) {
   static std::atomic<uint64_t> attr_devices{0};
-  auto kern = post_reduce_staged_kernel;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -872,7 +950,7 @@ cudaError_t launch_reduce_staged(const ElemArgs& a, cudaStream_t s) {
 
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
-  if (a.staged && !a.x_fp32 && !a.equilibrate) return launch_reduce_staged(a, s);
+  if (a.staged && !a.x_fp32 && !a.equilibrate) return launch_staged_impl<post_reduce_staged_kernel>(a, s);
   if (a.equilibrate)
     return a.x_fp32 ? launch_pdl(post_reduce_eq_kernel<true>, a.total_tiles, s, a)
                     : launch_pdl(post_reduce_eq_kernel<false>, a.total_tiles, s, a);
@@ -885,6 +963,7 @@ cudaError_t launch_post_finalize(const ElemArgs& a, cudaStream_t s) {
 }
 cudaError_t launch_post_apply(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
+  if (a.staged && !a.x_fp32 && !a.ns_only) return launch_staged_impl<post_apply_staged_kernel>(a, s);
   return a.x_fp32 ? launch_pdl(post_apply_kernel<true>, a.total_tiles, s, a)
                   : launch_pdl(post_apply_kernel<false>, a.total_tiles, s, a);
 }

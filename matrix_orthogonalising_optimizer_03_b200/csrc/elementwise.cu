@@ -901,6 +901,129 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
 
 // Launch with programmatic stream serialisation: the kernel may start while its
 // predecessor finishes and waits for it in griddep_wait().
+// ------------------------------------------------------------------ ingest (staged)
+// ingest with the G (bf16) and M loads staged in shared memory by cp.async, the ring of
+// the staged post-processing kernels with a stage of G (4 KB) and M (8 KB). M goes
+// back from the registers; U goes to the slab directly (wide) or through a bf16
+// transpose tile with the skewed rows of the staged reads (tall).
+constexpr int kStgInG = kTR * kTC * 2;               // G sub-tile (bf16), rows at 128 bytes
+constexpr int kStgInBytes = kStgInG + kTR * kTC * 4; // + M sub-tile, rows at 256 bytes
+constexpr int kStgInSmem = kStg * kStgInBytes + kStgO + 128;  // + the transpose tile
+static_assert(kStgInBytes % 128 == 0 && kStgO % 128 == 0, "stage alignment");
+
+__device__ __forceinline__ void stage_ingest(const DevMat& d, int r0, int c0, uint8_t* st) {
+  const int tid = threadIdx.x;
+  {  // G: 32 rows x 8 pieces of 8 bf16
+    const int row = tid >> 3, col = (tid & 7) * 8;
+    if (r0 + row < d.rows && c0 + col < d.cols)
+      cp_async16(st + row * (kTC * 2) + col * 2,
+                 static_cast<const uint16_t*>(d.G) + static_cast<int64_t>(r0 + row) * d.ld_g + c0 + col);
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {  // M: 32 rows x 16 pieces of 4 floats
+    const int q = tid + h * kThreads, row = q >> 4, col = (q & 15) * 4;
+    if (r0 + row < d.rows && c0 + col < d.cols)
+      cp_async16(st + kStgInG + row * (kTC * 4) + col * 4, d.M + static_cast<int64_t>(r0 + row) * d.ld_m + c0 + col);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 4) ingest_staged_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) &
+                                             ~static_cast<uintptr_t>(127));
+  uint8_t* tt = ring + kStg * kStgInBytes;  // tall: U transposed, skewed 64-byte rows
+  __shared__ double red[1][kThreads / 32];
+  const int b = blockIdx.x;
+  const int k = find_matrix(a, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const int t = b - a.tile_prefix[k];
+  const int sub_r = a.sub_r, sub_c = a.sub_c;
+  const int tiles_c = (d.cols + sub_c * kTC - 1) / (sub_c * kTC);
+  const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
+  const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
+  const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  const int nbr = min(sub_r, (d.rows - R0 + kTR - 1) / kTR);
+  const int nbc = min(sub_c, (d.cols - C0 + kTC - 1) / kTC);
+  const int nsub = nbr * nbc;
+  uint16_t* slab = static_cast<uint16_t*>(s.x0);
+#pragma unroll
+  for (int i = 0; i < kStg - 1; ++i) {
+    if (i < nsub) stage_ingest(d, R0 + (i % nbr) * kTR, C0 + (i / nbr) * kTC, ring + i * kStgInBytes);
+    cp_async_commit();
+  }
+  float sq = 0.f;
+  for (int i = 0; i < nsub; ++i) {
+    const int r0 = R0 + (i % nbr) * kTR, c0 = C0 + (i / nbr) * kTC;
+    const uint8_t* st = ring + (i % kStg) * kStgInBytes;
+    {
+      const int in = i + kStg - 1;
+      if (in < nsub) stage_ingest(d, R0 + (in % nbr) * kTR, C0 + (in / nbr) * kTC, ring + (in % kStg) * kStgInBytes);
+      cp_async_commit();
+    }
+    cp_async_wait<kStg - 1>();
+    __syncthreads();
+    const int r = r0 + lr, c = c0 + lc;
+    const int valid = r < d.rows ? max(0, min(8, d.cols - c)) : 0;
+    float u[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) u[e] = 0.f;
+    if (valid > 0) {
+      float g[8], m[8];
+      {
+        const uint4 gv = *reinterpret_cast<const uint4*>(st + lr * (kTC * 2) + lc * 2);
+        const uint32_t q[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          g[2 * e] = __uint_as_float(q[e] << 16);
+          g[2 * e + 1] = __uint_as_float(q[e] & 0xFFFF0000u);
+        }
+        const float4 x = *reinterpret_cast<const float4*>(st + kStgInG + lr * (kTC * 4) + lc * 4);
+        const float4 y = *reinterpret_cast<const float4*>(st + kStgInG + lr * (kTC * 4) + lc * 4 + 16);
+        m[0] = x.x; m[1] = x.y; m[2] = x.z; m[3] = x.w;
+        m[4] = y.x; m[5] = y.y; m[6] = y.z; m[7] = y.w;
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        m[e] = fmaf(a.mu, m[e], g[e]);                       // M_t = mu*M_{t-1} + G_t
+        u[e] = a.nesterov ? fmaf(a.mu, m[e], g[e]) : m[e];  // U = G_t + mu*M_t
+        if (e >= valid) u[e] = 0.f;
+      }
+      store8_f32(d.M + static_cast<int64_t>(r) * d.ld_m + c, true, valid, m);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {  // ||U|| of the slab's bf16 values
+      const float q = bf16_to_f32(f32_to_bf16(u[e]));
+      sq = fmaf(q, q, sq);
+    }
+    if (!tall) {
+      if (valid > 0) store8_bf16(slab + static_cast<int64_t>(r) * s.ldx + c, true, valid, u);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        *reinterpret_cast<uint16_t*>(tt + o_tall_off(lc + e) + lr * 2) = f32_to_bf16(u[e]);
+      __syncthreads();
+      const int k2 = threadIdx.x >> 2, col = (threadIdx.x & 3) * 8;  // slab row c0 + k2
+      const int v2 = c0 + k2 < d.cols ? max(0, min(8, d.rows - (r0 + col))) : 0;
+      if (v2 == 8) {
+        *reinterpret_cast<uint4*>(slab + static_cast<int64_t>(c0 + k2) * s.ldx + r0 + col) =
+            *reinterpret_cast<const uint4*>(tt + o_tall_off(k2) + col * 2);
+      } else {
+        for (int e = 0; e < v2; ++e)
+          slab[static_cast<int64_t>(c0 + k2) * s.ldx + r0 + col + e] =
+              *reinterpret_cast<const uint16_t*>(tt + o_tall_off(k2) + (col + e) * 2);
+      }
+    }
+    __syncthreads();  // the stage (and the transpose tile) are free again
+  }
+  cp_async_wait<0>();
+  double acc[1] = {sq};
+  block_sum<1>(acc, red);
+  if (threadIdx.x == 0) atomicAdd(&a.scal[k].u2, acc[0]);
+}
+
 template <typename... Args>
 cudaError_t launch_pdl(void (*kern)(Args...), unsigned grid, cudaStream_t s, const ElemArgs& a) {
   cudaLaunchConfig_t cfg = {};
@@ -916,14 +1039,9 @@ cudaError_t launch_pdl(void (*kern)(Args...), unsigned grid, cudaStream_t s, con
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
-  if (a.total_tiles <= 0) return cudaSuccess;
-  ingest_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
-  return cudaGetLastError();
-}
 // Shared-memory staged kernels: they need more than the default 48 KB of dynamic shared
 // memory; the opt-in is a per-device attribute, set once on each device (per kernel).
-template <void (*kern)(ElemArgs)>
+template <void (*kern)(ElemArgs), int kSmem = kStgSmem, bool kPdl = true>
 cudaError_t launch_staged_impl(const ElemArgs& a, cudaStream_t s) {
   static std::atomic<uint64_t> attr_devices{0};
   int dev = 0;
@@ -931,23 +1049,30 @@ cudaError_t launch_staged_impl(const ElemArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (uint64_t{1} << dev) : 0;
   if (bit == 0 || !(attr_devices.load(std::memory_order_acquire) & bit)) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStgSmem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     attr_devices.fetch_or(bit, std::memory_order_acq_rel);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.total_tiles, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kStgSmem;
+  cfg.dynamicSmemBytes = kSmem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = kPdl ? 1 : 0;
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
+  if (a.total_tiles <= 0) return cudaSuccess;
+  // the first kernel of a step: no programmatic overlap with what precedes it
+  if (a.staged_in) return launch_staged_impl<ingest_staged_kernel, kStgInSmem, false>(a, s);
+  ingest_kernel<<<a.total_tiles, kThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
   if (a.staged && !a.x_fp32 && !a.equilibrate) return launch_staged_impl<post_reduce_staged_kernel>(a, s);

@@ -32,6 +32,7 @@ struct ElemArgs {
   int32_t xs_from_u2;   // ns_steps == 0: the slab holds U, scale it by 1/(||U||+eps)
   int32_t sub_r, sub_c; // super-tile = sub_r x sub_c sub-tiles of 32 x 64 (1..4 each)
   int32_t staged;       // plain reduction through a shared-memory ring (aligned W rows, bf16 slab)
+  int32_t staged_in;    // ingest through the ring (also bf16 G with rows of 16-byte multiples)
 };
 
 cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s);

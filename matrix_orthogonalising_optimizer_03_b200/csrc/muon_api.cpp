@@ -65,7 +65,8 @@ struct muon_plan_s {
   std::vector<int32_t> tile_prefix;
   int64_t eq_total = 0;
   int sub_r = 4, sub_c = 4;  // elementwise super-tile in 32 x 64 sub-tiles
-  bool staged = false;       // staged (shared-memory ring) post_reduce
+  bool staged = false;       // staged (shared-memory ring) post_reduce and post_apply
+  bool staged_in = false;    // staged ingest
   size_t off_scal = 0, off_coef = 0, off_desc = 0, off_slabs = 0, off_tiles = 0;
   size_t off_eq_o2 = 0, off_eq_wo = 0, ws_bytes = 0;
   // cached per workspace pointer and device
@@ -268,6 +269,10 @@ void build_plan(muon_plan_s* p) {
   p->staged = !p->x_fp32 && p->sub_r * p->sub_c > 1;
   for (int i = 0; i < n; ++i)
     p->staged = p->staged && (p->dev[i].flags & MAT_VEC_OK) != 0 && p->dev[i].cols % 4 == 0;
+  // staged ingest: bf16 gradients whose rows are 16-byte multiples, and a momentum
+  p->staged_in = p->staged && !p->ns_only;
+  for (int i = 0; i < n; ++i)
+    p->staged_in = p->staged_in && (p->dev[i].flags & MAT_G_BF16) != 0 && p->dev[i].cols % 8 == 0;
   p->tile_prefix.assign(n + 1, 0);
   for (int i = 0; i < n; ++i) {
     const int64_t t = int64_t((p->dev[i].rows + tr - 1) / tr) * ((p->dev[i].cols + tc - 1) / tc);
@@ -594,6 +599,7 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
   ea.sub_r = p->sub_r;
   ea.sub_c = p->sub_c;
   ea.staged = p->staged ? 1 : 0;
+  ea.staged_in = p->staged_in ? 1 : 0;
 
   {
     ProfScope ps(p, stream);

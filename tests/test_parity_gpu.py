@@ -428,15 +428,16 @@ def test_single_cta_variable_width_tiles_ragged_m(env, m):
     H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs"), H.TOL_BF16)
 
 
-@pytest.mark.parametrize("cols_tail", [4, 3])
+@pytest.mark.parametrize("cols_tail", [8, 4, 3])
 def test_plain_reduction_large_ragged_step(env, cols_tail):
-    """A step above 4M elements with MuonGS (which needs <W,O>, ||W||^2 and ||O||^2):
-    with every row a multiple of 16 bytes (cols_tail 4) the sums are taken by the
-    shared-memory staged reduction, whose sub-tiles here end ragged in rows and columns
-    and include a tall (transposed) matrix; with one odd width (cols_tail 3) the plan falls
-    back to the register-staged kernel. 2 steps against the oracle."""
+    """A step above 4M elements with MuonGS (which needs <W,O>, ||W||^2 and ||O||^2).
+    Every width a multiple of 8 (cols_tail 8): ingest, the reduction and post_apply all
+    stage their loads in shared memory; a width that is a multiple of 4 only (cols_tail 4,
+    bf16 gradient rows not 16-byte multiples): ingest keeps its register-staged kernel; an
+    odd width (cols_tail 3): all three do. The sub-tiles end ragged in rows and columns
+    and include a tall (transposed) matrix. 2 steps against the oracle."""
     B, torch = env
-    shapes = [(1000, 2048 + cols_tail), (2052, 1000), (516, 1284)]
+    shapes = [(1000, 2048 + cols_tail), (2056, 1000), (516, 1288)]
     W0 = [H.seeded(r, c, 2300 + i, 0.02) for i, (r, c) in enumerate(shapes)]
     grads = [[H.seeded_bf16(r, c, 2400 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
              for t in range(2)]

@@ -462,8 +462,8 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
 // the ring (4 blocks x 4 stages of 12 KB), not by the registers that hold pending
 // loads. Used when every W row segment of the plan is 16-byte aligned (rows of 16-byte
 // multiples, 4 | cols), the slab is bf16 and the step has no equilibration (with the
-// per-row and per-column sums as well, the register-staged kernel above measured
-// faster). For tall matrices a stage holds 64 slab rows of 64 bytes (32 storage rows of
+// per-row and per-column sums as well, within 64 registers for 4 blocks per SM, a staged
+// variant measured slower than the register-staged kernel above). For tall matrices a stage holds 64 slab rows of 64 bytes (32 storage rows of
 // one storage column each), skewed by 16 bytes every 8 rows so that the column reads
 // below meet no bank conflict.
 constexpr int kStg = 4;                              // ring stages
@@ -526,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 4) post_reduce_staged_kernel(const E
   const int R0 = (t / tiles_c) * (sub_r * kTR), C0 = (t % tiles_c) * (sub_c * kTC);
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  const float xs = slab_scale(a, k);  // 1/(||U||+eps) when the slab holds U (no iteration)
   // sub-tiles of the super-tile inside the matrix, band by band (64 columns each)
   const int nbr = min(sub_r, (d.rows - R0 + kTR - 1) / kTR);
   const int nbc = min(sub_c, (d.cols - C0 + kTC - 1) / kTC);
@@ -586,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 4) post_reduce_staged_kernel(const E
     __syncthreads();
   }
   cp_async_wait<0>();
-  double acc[3] = {ww, wo, oo};
+  double acc[3] = {ww, (double)wo * xs, (double)oo * xs * xs};
   block_sum<3>(acc, red);
   if (threadIdx.x == 0) {
     atomicAdd(&a.scal[k].w2, acc[0]);
@@ -838,6 +839,7 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
   const int lr = threadIdx.x >> 3, lc = (threadIdx.x & 7) * 8;
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
   const MatCoef cf = a.coef[k];
+  const float xs = slab_scale(a, k);  // 1/(||U||+eps) when the slab holds U (no iteration)
   const int nbr = min(sub_r, (d.rows - R0 + kTR - 1) / kTR);
   const int nbc = min(sub_c, (d.cols - C0 + kTC - 1) / kTC);
   const int nsub = nbr * nbc;
@@ -886,7 +888,7 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
       const float rowf = (cf.axis & 1) ? a.eq_o2[s.eq_off + r] : 1.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        float f = rowf;
+        float f = xs * rowf;
         if ((cf.axis & 2) && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
         w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
       }

@@ -428,18 +428,26 @@ def test_single_cta_variable_width_tiles_ragged_m(env, m):
     H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs"), H.TOL_BF16)
 
 
-@pytest.mark.parametrize("cols_tail", [8, 4, 3])
-def test_plain_reduction_large_ragged_step(env, cols_tail):
+@pytest.mark.parametrize("cols_tail,ns_steps,eq", [(8, 5, False), (4, 5, False), (3, 5, False),
+                                                   (8, 0, False), (8, 5, True), (8, 0, True)])
+def test_large_ragged_step_staged_kernels(env, cols_tail, ns_steps, eq):
     """A step above 4M elements with MuonGS (which needs <W,O>, ||W||^2 and ||O||^2).
     Every width a multiple of 8 (cols_tail 8): ingest, the reduction and post_apply all
     stage their loads in shared memory; a width that is a multiple of 4 only (cols_tail 4,
     bf16 gradient rows not 16-byte multiples): ingest keeps its register-staged kernel; an
-    odd width (cols_tail 3): all three do. The sub-tiles end ragged in rows and columns
-    and include a tall (transposed) matrix. 2 steps against the oracle."""
+    odd width (cols_tail 3): all three do. With equilibration the reduction also takes
+    the per-row and per-column sums; with no Newton-Schulz iteration the slab holds U
+    and every kernel applies 1/(||U||+eps) itself. The sub-tiles end ragged in rows and
+    columns and include a tall (transposed) matrix. 2 steps against the oracle."""
     B, torch = env
     shapes = [(1000, 2048 + cols_tail), (2056, 1000), (516, 1288)]
     W0 = [H.seeded(r, c, 2300 + i, 0.02) for i, (r, c) in enumerate(shapes)]
     grads = [[H.seeded_bf16(r, c, 2400 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
              for t in range(2)]
-    gpu = H.run_steps(B, torch, W0, grads, H.gpu_hp(B, mode="muongs", wd=0.1), torch.bfloat16)
-    H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs", wd=0.1), H.TOL_BF16)
+    hp = H.gpu_hp(B, mode="muongs", wd=0.1, ns_steps=ns_steps, equilibrate=eq)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.bfloat16)
+    ohp = H.oracle_hp(mode="muongs", wd=0.1, ns_steps=ns_steps, equilibrate=eq)
+    if eq:
+        H.compare_runs_equilibrated(gpu, W0, grads, ohp, H.TOL_BF16)
+    else:
+        H.compare_runs(gpu, W0, grads, ohp, H.TOL_BF16)

@@ -438,9 +438,10 @@ def test_large_ragged_step_staged_kernels(env, cols_tail, ns_steps, eq):
     odd width (cols_tail 3): all three do. With equilibration the reduction also takes
     the per-row and per-column sums; with no Newton-Schulz iteration the slab holds U
     and every kernel applies 1/(||U||+eps) itself. The sub-tiles end ragged in rows and
-    columns and include a tall (transposed) matrix. 2 steps against the oracle."""
+    columns, include a tall (transposed) matrix, and two matrices smaller than one 32 x 64
+    sub-tile. 2 steps against the oracle."""
     B, torch = env
-    shapes = [(1000, 2048 + cols_tail), (2056, 1000), (516, 1288)]
+    shapes = [(1000, 2048 + cols_tail), (2056, 1000), (516, 1288), (17, 24), (40, 8)]
     W0 = [H.seeded(r, c, 2300 + i, 0.02) for i, (r, c) in enumerate(shapes)]
     grads = [[H.seeded_bf16(r, c, 2400 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
              for t in range(2)]

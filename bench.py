@@ -5,8 +5,9 @@ One step = one pass of the whole step (momentum, normalisation, 5 Newton-Schulz
 iterations, [equilibration], scale, projection / decay, update) over every matrix of
 a shape set, with weights, momenta and gradients resident in HBM. Prints one JSON
 line. The default shape set is the largest one that fits a GPU, the 1.5B dense set;
-the line also carries `per_set`, the same measurement for the other shape sets, and
-`sharded`, the ZeRO-1 sharded step over a one-rank NCCL group.
+the line also carries `per_set`, the same measurement for the other shape sets,
+`sharded`, the ZeRO-1 sharded step over a one-rank NCCL group, and `next_rows`: the
+MuonH and two-sided steps on the 400M shapes and the QK-Clip rescale.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload dense_1p5b]
   python bench.py --impl reference ...   # the float64 CPU oracle on host cores
@@ -50,6 +51,8 @@ def parse_args():
     ap.add_argument("--dist", default="sharded", choices=["sharded", "replica"],
                     help="multi-GPU mode: ZeRO-1 sharded step over NCCL, or independent replicas")
     ap.add_argument("--no-per-set", action="store_true", help="skip the other shape sets")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the MuonH, two-sided and QK-Clip measurements")
     ap.add_argument("--no-sharded", action="store_true",
                     help="skip the one-rank NCCL sharded measurement at N = 1")
     ap.add_argument("--run", type=int, default=0,
@@ -482,8 +485,11 @@ def measure_plan(B, w, run, args, dev, world: int, peaks, peak_src, seed: int, f
         "matrices": w.n_matrices if specs is None else len(specs),
         "params": w.n_params if specs is None else sum(s.rows * s.cols for s in specs),
         "mode": run.mode, "weight_decay": run.weight_decay, "equilibrate": run.equilibrate,
-        "ns_path": "fp32 CUDA cores" if w.ns_fp32 else "bf16 tcgen05",
-        **ns_rates(prof, w, args.steps, ms, peaks, specs),
+        "ns_path": ("none (two-sided normalisation)" if run.mode == "twosided"
+                    else "fp32 CUDA cores" if w.ns_fp32 else "bf16 tcgen05"),
+        **(ns_rates(prof, w, args.steps, ms, peaks, specs) if run.mode != "twosided" else
+           {"ns_tflops_step": None, "ns_frac_step": None, "ns_tflops_phases": None,
+            "ns_frac_phases": None, "ns_ms_per_step": 0.0}),
         "roofline": roofline(prof, w, peaks, peak_src, w.name if specs is None else None, ms,
                              clocks),
         "elementwise": elementwise_rates(prof, peaks),
@@ -617,6 +623,55 @@ def measure_sharded(B, w, run, args, dev, world: int, rank: int, peaks, peak_src
 PER_SET = [("gpt160m", 0), ("gpt400m", 0), ("gpt400m", 1), ("moe_1b", 0), ("single_128x256", 0),
            ("single_128x256", 1)]
 
+# The surveyed NEXT rows that run as kernels of their own, each timed like a shape set:
+# the MuonH retraction and the two-sided normalisation on the 400M shapes (MuonW is the
+# Muon + weight-decay run of the same set, and the ZeRO-1 step is the "sharded" record).
+NEXT_RUNS = [("gpt400m", "muonh", 0.0), ("gpt400m", "twosided", 0.0)]
+
+
+def measure_qk_clip(B, args, dev, peaks):
+    """QK-Clip: the per-head rescale of the query and key weights (the Moonlight review's
+    MuonClip; the loss-spike page's QK-Clip section) on the attention shapes of the 1.5B
+    dense set: 24 layers of W_q and W_k, 2048 x 2048 fp32, 16 heads of 128 rows, with the
+    caller's S_max drawn so that half of the heads exceed tau = 100 (gamma = 2/3,
+    power 1/2 on each side). Algorithmic bytes: 8 per rescaled element (read and write);
+    heads at or below tau are not touched. Timed with CUDA events on the launching
+    stream over K calls of a QkClipPlan (descriptors marshalled once) after W warm-up
+    calls."""
+    import torch
+    layers, heads, d, hd = 24, 16, 2048, 128
+    g = torch.Generator(device=dev)
+    g.manual_seed(20)
+    wq = [torch.randn(d, d, device=dev, generator=g) * 0.02 for _ in range(layers)]
+    wk = [torch.randn(d, d, device=dev, generator=g) * 0.02 for _ in range(layers)]
+    hot = torch.rand(layers * heads, device=dev, generator=g) < 0.5
+    s_max = torch.where(hot, torch.full_like(hot, 150.0, dtype=torch.float32),
+                        torch.full_like(hot, 50.0, dtype=torch.float32))
+    slices = []
+    for li in range(layers):
+        for h in range(heads):
+            slices.append((wq[li], h * hd, hd, li * heads + h, 0.5))
+            slices.append((wk[li], h * hd, hd, li * heads + h, 0.5))
+    clip = B.QkClipPlan(slices, s_max, tau=100.0)  # the descriptors marshalled once
+    for _ in range(args.warmup):
+        clip.apply()
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        clip.apply()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    scaled = int(hot.sum().item()) * 2 * hd * d
+    gbs = 8.0 * scaled / (ms / 1e3) / 1e9
+    return {"ms_per_call": ms, "heads_clipped": int(hot.sum().item()),
+            "heads": layers * heads, "rescaled_elements": scaled,
+            "gb_s": gbs, "frac": gbs / peaks["hbm_gbs"], "bound": "hbm",
+            "what": "24 layers x (W_q, W_k) 2048 x 2048 fp32, 16 heads of 128 rows, "
+                    "half of the heads above tau"}
+
 
 # ------------------------------------------------------------------ GPU arm
 def main():
@@ -707,6 +762,17 @@ def main():
                 per[f"{name}/{ws.runs[ridx].mode}" + ("+wd" if ws.runs[ridx].weight_decay else "")] = r
                 torch.cuda.empty_cache()
             extra["per_set"] = per
+        if world == 1 and not args.no_next:
+            nxt = {}
+            for name, mode, wd in NEXT_RUNS:
+                ws = wl.WORKLOADS[name]
+                r, _, _ = measure_plan(B, ws, wl.Run(mode, wd), args, dev, 1, peaks, peak_src, 0,
+                                       full=False)
+                nxt[f"{mode}/{name}"] = r
+                torch.cuda.empty_cache()
+            nxt["qk_clip"] = measure_qk_clip(B, args, dev, peaks)
+            torch.cuda.empty_cache()
+            extra["next_rows"] = nxt
 
     if rank == 0:
         line = {

@@ -263,7 +263,8 @@ MUON_API muon_status_t muon_newton_schulz_noalloc(const muon_ns_matrix_t* mat,
  * `cols` columns, leading dimension ld) that belong to head `head` and are scaled by
  * gamma_head^power (0.5 or 1.0 in the listing). s_max_dev: device array of n_heads
  * floats (the caller's forward pass measures them). Slices of one call may not
- * overlap (MUON_ERR_ALIAS). Asynchronous on `stream`; no workspace. */
+ * overlap (MUON_ERR_ALIAS; a slice of zero rows overlaps nothing). cols is at most
+ * 2^26 (MUON_ERR_SHAPE). Asynchronous on `stream`; no workspace. */
 typedef struct {
   void* W;
   int64_t row0, rows, cols, ld;

@@ -348,21 +348,38 @@ def newton_schulz_noalloc(x, o, hp: MuonHParams, status=None, stream=None):
                                               _stream_ptr(stream)), "muon_newton_schulz_noalloc")
 
 
+class QkClipPlan:
+    """QK-Clip over a fixed set of slices: the slice descriptors are marshalled once, and
+    every `apply()` rescales the heads whose current S_max (read on the device from the
+    same `s_max` tensor) exceeds tau. slices: list of (W tensor fp32 2-D CUDA, row0, rows,
+    head, power); s_max: CUDA float32 tensor with one entry per head. The weights and
+    s_max must stay alive while the plan is used."""
+
+    def __init__(self, slices, s_max, tau: float = 100.0):
+        self._lib = load()
+        arr = (MuonQkSlice * len(slices))()
+        for i, (w, r0, nr, h, pw) in enumerate(slices):
+            _check_2d(w, "W")
+            if w.dtype != _torch().float32:
+                raise MuonError(3, "QK-Clip weights must be float32")
+            if w.device != s_max.device:
+                raise MuonError(1, "QK-Clip weights and s_max must be on the same GPU")
+            arr[i] = MuonQkSlice(w.data_ptr(), r0, nr, w.size(1), max(w.stride(0), w.size(1)), h, pw)
+        if s_max.dtype != _torch().float32 or not s_max.is_cuda:
+            raise MuonError(1, "s_max must be a CUDA float32 tensor")
+        self._arr, self._n, self.s_max, self.tau = arr, len(slices), s_max, float(tau)
+
+    def apply(self, stream=None):
+        with _on(self.s_max.device):
+            _check(self._lib.muon_qk_clip(self._arr, self._n, self.s_max.data_ptr(),
+                                          self.s_max.numel(), self.tau, _stream_ptr(stream)),
+                   "muon_qk_clip")
+
+
 def qk_clip(slices, s_max, tau: float = 100.0, stream=None):
-    """QK-Clip. slices: list of (W tensor fp32 2-D CUDA, row0, rows, head, power);
+    """QK-Clip, one call. slices: list of (W tensor fp32 2-D CUDA, row0, rows, head, power);
     s_max: CUDA float32 tensor with one entry per head."""
-    lib = load()
-    arr = (MuonQkSlice * len(slices))()
-    for i, (w, r0, nr, h, pw) in enumerate(slices):
-        _check_2d(w, "W")
-        if w.dtype != _torch().float32:
-            raise MuonError(3, "QK-Clip weights must be float32")
-        arr[i] = MuonQkSlice(w.data_ptr(), r0, nr, w.size(1), max(w.stride(0), w.size(1)), h, pw)
-    if s_max.dtype != _torch().float32 or not s_max.is_cuda:
-        raise MuonError(1, "s_max must be a CUDA float32 tensor")
-    with _on(s_max.device):
-        _check(lib.muon_qk_clip(arr, len(slices), s_max.data_ptr(), s_max.numel(), tau,
-                                _stream_ptr(stream)), "muon_qk_clip")
+    QkClipPlan(slices, s_max, tau).apply(stream)
 
 
 class StreamedSteps:

@@ -177,14 +177,20 @@ __device__ __forceinline__ void cluster_phase_barrier() {
 
 // Fused kernel tile: a 32 x 32 (GRAM, POLY) or 32 x 64 (APPLY) output tile computed from
 // full-K operand panels staged in shared memory by one round of loads (K <= kFusedMaxK),
-// so that the tile pays the L2 latency once instead of once per k-step. 2 x 2 (2 x 4)
-// outputs per thread, in k order.
-//   As[i][k] = A[i0 + i][k]                      (row stride kFusedStride, odd)
+// so that the tile pays the L2 latency once instead of once per k-step. 128 threads
+// compute, each a 4 x 2 (GRAM, POLY) or 4 x 4 (APPLY) block of outputs from 16-byte
+// reads of both panels along k (4 k-steps per read), each output one fp32 dot product
+// in k order.
+//   As[i][k] = A[i0 + i][k]                      (row stride kFusedStride)
 //   GRAM / POLY: Bs[j][k] = B[j0 + j][k]         (B is X, or S, which is symmetric)
 //   APPLY:       Bs[k][j] = X[k][j0 + j]          (row stride 64)
+// kFusedStride is a multiple of 4 (16-byte rows) whose rows are 16 bytes apart modulo
+// 128: the reads of 8 consecutive rows at one k fall in different banks.
 constexpr int kFusedMaxK = 256;
-constexpr int kFusedStride = kFusedMaxK + 1;  // odd row stride: conflict-free column reads
+constexpr int kFusedStride = kFusedMaxK + 4;
 constexpr int kApplyTN = 64;                  // APPLY tile columns
+constexpr int kFusedMathThreads = 128;
+static_assert((kFusedStride * 4) % 128 == 16, "panel rows 16 bytes apart modulo 128");
 
 template <int PHASE>
 __device__ __forceinline__ void fused_tile(const NsClassArgs& k, int mat, int t, const float* X,
@@ -271,56 +277,69 @@ __device__ __forceinline__ void fused_tile(const NsClassArgs& k, int mat, int t,
         if (kk < K) *reinterpret_cast<float2*>(Bs + kk * kApplyTN + 2 * lane) = v[q];
       }
     }
+    // rows K .. K rounded up to 4 are read (times a zero of A): keep them finite
+    for (int kk = K + warp; kk < ((K + 3) & ~3); kk += NT / 32)
+      *reinterpret_cast<float2*>(Bs + kk * kApplyTN + 2 * lane) = make_float2(0.f, 0.f);
   }
   __syncthreads();
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  constexpr int NY = PHASE == PH_APPLY ? 4 : 2;  // output columns per thread
-  float acc[2][NY];
+  if (threadIdx.x < kFusedMathThreads) {
+    // rows ty + 8i (i < 4); columns tx + 16j (j < 2: GRAM, POLY) or 4tx .. 4tx + 3 (APPLY)
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    constexpr int NY = PHASE == PH_APPLY ? 4 : 2;
+    const int K4 = (K + 3) & ~3;  // panel entries past K are 0 in A (and finite in B)
+    float acc[4][NY];
 #pragma unroll
-  for (int x = 0; x < 2; ++x)
+    for (int x = 0; x < 4; ++x)
 #pragma unroll
-    for (int y = 0; y < NY; ++y) acc[x][y] = 0.f;
-  const float* a0 = As + (ty * 2) * kFusedStride;
-  const float* a1 = a0 + kFusedStride;
-  if (PHASE == PH_APPLY) {
-    for (int kk = 0; kk < K; ++kk) {
-      const float av[2] = {a0[kk], a1[kk]};
-      const float4 bq = *reinterpret_cast<const float4*>(Bs + kk * kApplyTN + tx * 4);
-      const float bv[4] = {bq.x, bq.y, bq.z, bq.w};
+      for (int y = 0; y < NY; ++y) acc[x][y] = 0.f;
+    for (int kk = 0; kk < K4; kk += 4) {
+      float av[4][4];
 #pragma unroll
-      for (int x = 0; x < 2; ++x)
+      for (int x = 0; x < 4; ++x) {
+        const float4 q = *reinterpret_cast<const float4*>(As + (ty + 8 * x) * kFusedStride + kk);
+        av[x][0] = q.x; av[x][1] = q.y; av[x][2] = q.z; av[x][3] = q.w;
+      }
+      float bv[4][NY];  // [k offset][column]
+      if (PHASE == PH_APPLY) {
 #pragma unroll
-        for (int y = 0; y < NY; ++y) acc[x][y] = fmaf(av[x], bv[y], acc[x][y]);
-    }
-  } else {
-    const float* b0 = Bs + (tx * 2) * kFusedStride;
-    const float* b1 = b0 + kFusedStride;
-    for (int kk = 0; kk < K; ++kk) {
-      const float av0 = a0[kk], av1 = a1[kk], bv0 = b0[kk], bv1 = b1[kk];
-      acc[0][0] = fmaf(av0, bv0, acc[0][0]);
-      acc[0][1] = fmaf(av0, bv1, acc[0][1]);
-      acc[1][0] = fmaf(av1, bv0, acc[1][0]);
-      acc[1][1] = fmaf(av1, bv1, acc[1][1]);
-    }
-  }
-#pragma unroll
-  for (int x = 0; x < 2; ++x) {
-    const int i = i0 + ty * 2 + x;
-    if (i >= m) continue;
-#pragma unroll
-    for (int y = 0; y < NY; ++y) {
-      const int j = j0 + tx * NY + y;
-      if (j >= ncols) continue;
-      if (PHASE == PH_GRAM) {
-        const float v = scale * acc[x][y];
-        Sw[(int64_t)i * k.lds + j] = v;
-        if (ti != tj) Sw[(int64_t)j * k.lds + i] = v;
-      } else if (PHASE == PH_POLY) {
-        const float v = fmaf(pb, S[(int64_t)i * k.lds + j], pc * acc[x][y]);
-        Pm[(int64_t)i * k.lds + j] = v;
-        if (ti != tj) Pm[(int64_t)j * k.lds + i] = v;
+        for (int e = 0; e < 4; ++e) {
+          const float4 q = *reinterpret_cast<const float4*>(Bs + (kk + e) * kApplyTN + 4 * tx);
+          bv[e][0] = q.x; bv[e][1] = q.y;
+          bv[e][NY > 2 ? 2 : 0] = q.z; bv[e][NY > 3 ? 3 : 0] = q.w;
+        }
       } else {
-        Xout[(int64_t)i * k.ldx + j] = scale * fmaf(pa, X[(int64_t)i * k.ldx + j], acc[x][y]);
+#pragma unroll
+        for (int y = 0; y < NY; ++y) {
+          const float4 q = *reinterpret_cast<const float4*>(Bs + (tx + 16 * y) * kFusedStride + kk);
+          bv[0][y] = q.x; bv[1][y] = q.y; bv[2][y] = q.z; bv[3][y] = q.w;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e)  // k order
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < NY; ++y) acc[x][y] = fmaf(av[x][e], bv[e][y], acc[x][y]);
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int i = i0 + ty + 8 * x;
+      if (i >= m) continue;
+#pragma unroll
+      for (int y = 0; y < NY; ++y) {
+        const int j = j0 + (PHASE == PH_APPLY ? 4 * tx + y : tx + 16 * y);
+        if (j >= ncols) continue;
+        if (PHASE == PH_GRAM) {
+          const float v = scale * acc[x][y];
+          Sw[(int64_t)i * k.lds + j] = v;
+          if (ti != tj) Sw[(int64_t)j * k.lds + i] = v;
+        } else if (PHASE == PH_POLY) {
+          const float v = fmaf(pb, S[(int64_t)i * k.lds + j], pc * acc[x][y]);
+          Pm[(int64_t)i * k.lds + j] = v;
+          if (ti != tj) Pm[(int64_t)j * k.lds + i] = v;
+        } else {
+          Xout[(int64_t)i * k.ldx + j] = scale * fmaf(pa, X[(int64_t)i * k.ldx + j], acc[x][y]);
+        }
       }
     }
   }

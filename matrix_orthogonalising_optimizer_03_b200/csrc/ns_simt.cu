@@ -169,9 +169,10 @@ __global__ void __launch_bounds__(NT) ns_simt_kernel(const NsPhaseArgs p) {
                              p.c, As, Bs);
 }
 
-// Release this block's global stores and wait for every block of the cluster.
+// Release this block's global stores and wait for every block of the cluster. Every
+// reader of a phase's output is a thread of the same cluster, so the barrier's release /
+// acquire at cluster scope orders the stores for them (no device-scope fence).
 __device__ __forceinline__ void cluster_phase_barrier() {
-  __threadfence();
   cluster_sync_all();
 }
 

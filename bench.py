@@ -176,9 +176,10 @@ def traffic_record(kernel: str, workload: str):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def oracle_sample(w, run, budget_s: float, rotate: int = 0):
+def oracle_sample(w, run, budget_s: float, rotate: int = 0, smallest_only: bool = False):
     """Times the float64 oracle on a stratified sample of the shape set and extrapolates
-    to one full step: sum over shape classes of count x mean seconds per matrix."""
+    to one full step: sum over shape classes of count x mean seconds per matrix. With
+    `smallest_only` (warm-up) it runs one matrix of the smallest shape class."""
     from matrix_orthogonalising_optimizer_03_b200 import workloads as wl
     from oracle import muon_oracle as orc
     hp = orc.HParams(lr=w.lr, momentum=w.momentum, weight_decay=run.weight_decay, mode=run.mode,
@@ -187,6 +188,9 @@ def oracle_sample(w, run, budget_s: float, rotate: int = 0):
     by_class = {}
     for s in specs:
         by_class.setdefault((s.rows, s.cols), []).append(s)
+    if smallest_only:
+        key = min(by_class, key=lambda k: k[0] * k[1])
+        by_class = {key: by_class[key]}
     t_start = time.perf_counter()
     per_class, sampled = {}, 0
     rounds = 0
@@ -223,8 +227,8 @@ def run_reference(args, rank: int, world: int):
     w = wl.WORKLOADS[args.workload]
     run = w.runs[args.run]
     per_step = max(1.0, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
-    for i in range(args.warmup):
-        oracle_sample(w, run, 0.0, rotate=i)
+    for i in range(args.warmup):  # untimed; one small matrix pages the code in
+        oracle_sample(w, run, 0.0, rotate=i, smallest_only=True)
     times, sampled = [], 0
     for i in range(args.steps):
         est, n, _ = oracle_sample(w, run, per_step, rotate=args.warmup + i)

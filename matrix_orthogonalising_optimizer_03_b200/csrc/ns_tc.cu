@@ -25,18 +25,22 @@
 // which lands chunk after chunk in the MN-major layout.
 //
 // Kernel structure (persistent, one CTA per SM, 320 threads):
-//   warp 0     TMA producer: a STAGES-deep ring of 128B-swizzled shared-memory
-//              stages; every load lands in one CTA's own shared memory.
+//   warp 0     TMA producer: a ring of 128B-swizzled shared-memory stages (as many as
+//              fit 224 KB; single-CTA symmetric launches size their stages to their
+//              largest tile); every load lands in one CTA's own shared memory. On the
+//              block diagonal of GRAM and POLY it loads B only (A is B's first rows).
 //   warp 1     TMEM allocator and MMA issuer (one thread), double-buffered fp32
 //              accumulator in TMEM.
 //   warps 2-9  epilogue: two warps per TMEM lane quarter, each taking every other
 //              64-column chunk; tcgen05.ld, fused scale / polynomial, and per warp a
 //              32 x 64 bf16 box staged in swizzled shared memory and written with the
 //              warp's own TMA store (which clips ragged edges), with no barrier between
-//              the warps. POLY's C tile (S) arrives by TMA one tile ahead.
+//              the warps. POLY's C tile (S) arrives by TMA one tile ahead (CTA pairs)
+//              or is read from L2 into registers (single CTA).
 // Two variants:
-//   single CTA   tile 128 x BN (BN = 128 for GRAM / POLY, 256 for APPLY),
-//                tcgen05.mma.cta_group::1, M = 128.
+//   single CTA   APPLY tiles 128 x 256; GRAM / POLY tiles of one 128-row block and a
+//                variable-width column piece (sym_piece), described stage by stage by
+//                the producer to the MMA issuer; tcgen05.mma.cta_group::1, M = 128.
 //   CTA pair     cluster of two CTAs, tile 256 x 256, tcgen05.mma.cta_group::2
 //                (M = N = 256): each CTA loads its 128 rows of A and half of B into
 //                its own shared memory (plain TMA loads whose bytes count on the first

@@ -198,3 +198,17 @@ def test_noalloc_binding_rejects_bad_status_before_any_launch(lib):
         with pytest.raises(B.MuonError) as e:
             B.newton_schulz_noalloc(x, o, hp, status=status)
         assert e.value.status == 1 and "status" in str(e.value)
+
+
+def test_qk_clip_plan_rejects_bad_inputs_before_any_launch(lib):
+    """QkClipPlan checks its slices and S_max on the host: host-memory weights, weights of
+    another dtype or layout, and a host S_max raise MuonError before the library is
+    called."""
+    import torch
+    s_dev = _FakeCudaTensor(torch.float32, 4)
+    bad = [[(torch.zeros(8, 8), 0, 4, 0, 0.5)],                       # host weights
+           [(torch.zeros(2, 8, 8), 0, 4, 0, 0.5)],                    # not 2-D
+           [(torch.zeros(8, 8).t()[:, :4], 0, 4, 0, 0.5)]]            # column-major view
+    for slices in bad:
+        with pytest.raises(B.MuonError):
+            B.QkClipPlan(slices, s_dev)

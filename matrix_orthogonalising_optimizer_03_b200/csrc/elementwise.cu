@@ -455,17 +455,18 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
 }
 
 // ------------------------------------------------------------------ post_reduce (staged)
-// The three per-matrix sums with the loads moved out of the registers: every thread copies its
-// share of each 32 x 64 sub-tile (W rows and slab rows, 16 bytes per copy) into a ring of
-// shared-memory stages with cp.async, kStg - 1 sub-tiles ahead of the arithmetic, and
-// reads its 8 elements back from shared memory. Bytes in flight per SM are then set by
-// the ring (4 blocks x 4 stages of 12 KB), not by the registers that hold pending
-// loads. Used when every W row segment of the plan is 16-byte aligned (rows of 16-byte
-// multiples, 4 | cols), the slab is bf16 and the step has no equilibration (with the
-// per-row and per-column sums as well, within 64 registers for 4 blocks per SM, a staged
-// variant measured slower than the register-staged kernel above). For tall matrices a stage holds 64 slab rows of 64 bytes (32 storage rows of
+// The three per-matrix sums with the loads moved out of the registers: every thread
+// copies its share of each 32 x 64 sub-tile (W rows and slab rows, 16 bytes per copy)
+// into a ring of shared-memory stages with cp.async, kStg - 1 sub-tiles ahead of the
+// arithmetic, and reads its 8 elements back from shared memory. Bytes in flight per SM
+// are then set by the ring (4 blocks x 4 stages of 12 KB), not by the registers that
+// hold pending loads. Used when every W row segment of the plan is 16-byte aligned
+// (rows of 16-byte multiples, 4 | cols), the slab is bf16 and the step has no
+// equilibration (with the per-row and per-column sums as well, within 64 registers for
+// 4 blocks per SM, a staged variant measured slower than the register-staged kernel
+// above). For tall matrices a stage holds 64 slab rows of 64 bytes (32 storage rows of
 // one storage column each), skewed by 16 bytes every 8 rows so that the column reads
-// below meet no bank conflict.
+// below meet no bank conflict. post_apply and ingest use the same ring.
 constexpr int kStg = 4;                              // ring stages
 constexpr int kStgW = kTR * kTC * 4;                 // W sub-tile, rows at 256 bytes
 constexpr int kStgO = kTC * kTR * 2 + 8 * 16;        // O sub-tile (tall: skewed rows)

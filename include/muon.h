@@ -205,11 +205,13 @@ MUON_API muon_status_t muon_newton_schulz_batched(const muon_ns_matrix_t* mats, 
 /* ---- per-kernel device timing of a plan (CUDA events around each launch) ----
  * Kernel kinds: "ingest", "ns_gram", "ns_poly", "ns_apply", "post_reduce",
  * "post_finalize", "post_apply", "ns_fused" (the fp32 path's single launch over all
- * iterations of small matrices). flops / bytes are the algorithmic work of the
+ * iterations of small matrices), "post_stats" (the statistics of MUON_MODE_MUON and
+ * MUON_MODE_TWOSIDED, after post_apply). flops / bytes are the algorithmic work of the
  * recorded launches: Newton-Schulz flops count the symmetric Gram and polynomial
  * once (m(m+1)n and m^2(m+1)) and the apply 2m^2n; bytes count each kernel's own
  * inputs and outputs once (ingest: G, M read, M and X_0 written; post_reduce: W and
- * O read; post_apply: W read and written, O read). */
+ * O read, or O alone in MUON_MODE_MUON and MUON_MODE_TWOSIDED, whose update needs no
+ * scalar of W; post_apply: W read and written, O read). */
 typedef struct {
   char name[32];
   int32_t launches;   /* launches recorded since the last read */

@@ -5,10 +5,14 @@
 //                 (transposed through shared memory for tall matrices).
 //   post_reduce   ||W||^2, <W,O>, ||O||^2 (post_reduce_plain_kernel); with
 //                 equilibration also per-row and per-column sums of O^2 and W*O in the
-//                 storage frame (post_reduce_eq_kernel).
+//                 storage frame (post_reduce_eq_kernel). Muon and the two-sided mode
+//                 need no W-dependent scalar: ||O||^2 and the O^2 row / column sums
+//                 from the slab alone (post_reduce_o_kernel).
 //   post_finalize one block per matrix: equilibration axis and factors (a6),
 //                 scale (a7), GS coefficient (a8), statistics, update coefficients.
-//   post_apply    a9: W <- cw*W + co*D*O (or, Newton-Schulz only, O out).
+//   post_apply    a9: W <- cw*W + co*D*O (or, Newton-Schulz only, O out); in Muon and
+//                 the two-sided mode also the statistics' sums of W_t and D*O.
+//   post_stats    statistics of Muon and the two-sided mode (one thread per matrix).
 //
 // Work unit: a 128 x 256 super-tile of the matrix in its storage frame per
 // 256-thread block, walked as 4 x 4 sub-tiles of 32 x 64 (8 consecutive columns
@@ -116,13 +120,16 @@ __device__ __forceinline__ void block_sum(double (&v)[NV], double (*sh)[kThreads
   }
 }
 
-__device__ __forceinline__ int find_matrix(const ElemArgs& a, int b) {
-  int lo = 0, hi = a.n - 1;
+__device__ __forceinline__ int find_matrix_in(const int32_t* prefix, int n, int b) {
+  int lo = 0, hi = n - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(a.tile_prefix + mid) <= b) lo = mid; else hi = mid - 1;
+    if (__ldg(prefix + mid) <= b) lo = mid; else hi = mid - 1;
   }
   return lo;
+}
+__device__ __forceinline__ int find_matrix(const ElemArgs& a, int b) {
+  return find_matrix_in(a.tile_prefix, a.n, b);
 }
 
 // ------------------------------------------------------------------ ingest
@@ -454,6 +461,164 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
   }
 }
 
+// ------------------------------------------------------------------ post_reduce (O only)
+// Muon and the two-sided mode: ||O||^2 and the per-row and per-column sums of O^2,
+// read from the Newton-Schulz slab alone (2 bytes per element in bf16) in the slab's
+// own frame, where a slab row is a W row (wide) or a W column (tall: the slab holds
+// O^T), so nothing is transposed. A block takes a band of kOTileR slab rows across the
+// whole width, in kOTileC-column tiles: each warp 8 rows, each lane 8 consecutive
+// columns of a tile (eight 16-byte loads, two each in fp32, issued before the
+// arithmetic). In bf16 4 blocks per SM (64 registers) keep loads in flight while a
+// block sums; two register buffers with the next tile's loads issued ahead (2 blocks
+// per SM) measured 14 % slower. A tile's column partials are summed over the 8 warps
+// through double-buffered shared memory (one barrier per tile) and flushed with one
+// atomic per column; the row partials stay in registers over the band and are summed
+// over the warp at its end by a halving exchange (each step keeps half of the rows and
+// adds the partner's half: 4 + 2 + 1 shuffles, then 2 to finish). Slab columns past n
+// hold whatever the Newton-Schulz stores left there and are masked.
+template <bool XF32>
+struct OTileRegs;
+template <>
+struct OTileRegs<false> {
+  uint4 q[8];
+};
+template <>
+struct OTileRegs<true> {
+  float4 q[8][2];
+};
+
+template <bool XF32>
+__device__ __forceinline__ void o_tile_load(OTileRegs<XF32>& b, const void* slab, int64_t ldx, int rw,
+                                            int sm, int c, int sn) {
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const bool in = c < sn && rw + p < sm;
+    if constexpr (XF32) {
+      b.q[p][0] = b.q[p][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (in) {
+        const float4* src =
+            reinterpret_cast<const float4*>(static_cast<const float*>(slab) + (rw + p) * ldx + c);
+        b.q[p][0] = __ldcs(src);
+        b.q[p][1] = __ldcs(src + 1);
+      }
+    } else {
+      b.q[p] = make_uint4(0u, 0u, 0u, 0u);
+      if (in)
+        b.q[p] = __ldcs(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(slab) + (rw + p) * ldx + c));
+    }
+  }
+}
+
+// rp[p] += sum over the lane's valid columns of row p; cp[e] += sum over the 8 rows
+template <bool XF32>
+__device__ __forceinline__ void o_tile_sums(const OTileRegs<XF32>& b, int nv, float (&rp)[8],
+                                            float (&cp)[8]) {
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    float v[8];
+    if constexpr (XF32) {
+      v[0] = b.q[p][0].x; v[1] = b.q[p][0].y; v[2] = b.q[p][0].z; v[3] = b.q[p][0].w;
+      v[4] = b.q[p][1].x; v[5] = b.q[p][1].y; v[6] = b.q[p][1].z; v[7] = b.q[p][1].w;
+    } else {
+      const uint32_t w4[4] = {b.q[p].x, b.q[p].y, b.q[p].z, b.q[p].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __uint_as_float(w4[e] << 16);
+        v[2 * e + 1] = __uint_as_float(w4[e] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float x = e < nv ? v[e] : 0.f;
+      rp[p] = fmaf(x, x, rp[p]);
+      cp[e] = fmaf(x, x, cp[e]);
+    }
+  }
+}
+
+template <bool XF32>
+__global__ void __launch_bounds__(kThreads, XF32 ? 2 : 4) post_reduce_o_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  static_assert(kOTileR == 8 * (kThreads / 32) && kOTileC == 8 * 32 && kOTileC == kThreads,
+                "8 rows per warp, 8 columns per lane, one column per thread");
+  __shared__ __align__(16) float colsh[2][kThreads / 32][kOTileC];
+  __shared__ double red[1][kThreads / 32];
+  const int b = blockIdx.x;
+  const int k = find_matrix_in(a.o_tile_prefix, a.n, b);
+  const DevMat d = a.mats[k];
+  const DevSlab s = a.slabs[k];
+  const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
+  const int sm = tall ? d.cols : d.rows, sn = tall ? d.rows : d.cols;  // slab rows, cols
+  const int R0 = (b - a.o_tile_prefix[k]) * kOTileR;
+  const int ntc = (sn + kOTileC - 1) / kOTileC;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rw = R0 + warp * 8;
+  const float xs = slab_scale(a, k);
+  const float xs2 = xs * xs;
+  float* col_out = a.eq_o2 + s.eq_off + (tall ? 0 : d.rows);  // W rows (tall) or W columns
+  float rp[8];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) rp[p] = 0.f;
+  // c + 8 <= ldx whenever c < sn (ldx is a multiple of 64), so a whole 8-group load
+  // stays inside the slab row
+  auto tile = [&](const OTileRegs<XF32>& buf, int j) {
+    const int c = j * kOTileC + lane * 8;
+    float cp[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cp[e] = 0.f;
+    o_tile_sums<XF32>(buf, max(0, min(8, sn - c)), rp, cp);
+    float4* dst = reinterpret_cast<float4*>(&colsh[j & 1][warp][lane * 8]);
+    dst[0] = make_float4(cp[0], cp[1], cp[2], cp[3]);
+    dst[1] = make_float4(cp[4], cp[5], cp[6], cp[7]);
+    __syncthreads();  // the buffer of tile j + 2 is written after the next barrier
+    float col = 0.f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) col += colsh[j & 1][w][threadIdx.x];
+    const int cc = j * kOTileC + threadIdx.x;
+    if (cc < sn) atomicAdd(col_out + cc, col * xs2);
+  };
+  {
+    OTileRegs<XF32> A;
+    for (int j = 0; j < ntc; ++j) {
+      o_tile_load<XF32>(A, s.xf, s.ldx, rw, sm, j * kOTileC + lane * 8, sn);
+      tile(A, j);
+    }
+  }
+  float tot = 0.f;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) tot += rp[p];
+  // row sums over the warp: after the exchanges on lane bits 4, 3 and 2 each lane holds
+  // row (lane >> 2) & 7 summed over 8 lanes; bits 1 and 0 finish the sum
+  float h4[4], h2[2];
+  const bool b4 = (lane & 16) != 0, b3 = (lane & 8) != 0, b2 = (lane & 4) != 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float keep = b4 ? rp[i + 4] : rp[i], give = b4 ? rp[i] : rp[i + 4];
+    h4[i] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const float keep = b3 ? h4[i + 2] : h4[i], give = b3 ? h4[i] : h4[i + 2];
+    h2[i] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+  }
+  float row;
+  {
+    const float keep = b2 ? h2[1] : h2[0], give = b2 ? h2[0] : h2[1];
+    row = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+  }
+  row += __shfl_xor_sync(0xffffffffu, row, 2);
+  row += __shfl_xor_sync(0xffffffffu, row, 1);
+  {
+    const int r = rw + ((lane >> 2) & 7);
+    if ((lane & 3) == 0 && r < sm)
+      atomicAdd(a.eq_o2 + s.eq_off + (tall ? d.rows + r : r), row * xs2);
+  }
+  double acc[1] = {tot};
+  block_sum<1>(acc, red);
+  if (threadIdx.x == 0) atomicAdd(&a.scal[k].o2, acc[0] * xs2);
+}
+
 // ------------------------------------------------------------------ post_reduce (staged)
 // The three per-matrix sums with the loads moved out of the registers: every thread
 // copies its share of each 32 x 64 sub-tile (W rows and slab rows, 16 bytes per copy)
@@ -610,6 +775,14 @@ __device__ __forceinline__ double block_sum2(double& x, double& y, double (*sh)[
   return x;
 }
 
+// a7: the scale s of the orthogonalised update
+__device__ __forceinline__ double step_scale(const ElemArgs& a, const DevMat& d) {
+  const double rows = d.rows, cols = d.cols;
+  if (a.scale_rule == MUON_SCALE_MOONLIGHT) return (double)a.scale_k * sqrt(fmax(rows, cols));
+  if (a.scale_rule == MUON_SCALE_KELLER) return sqrt(fmax(1.0, rows / cols));
+  return 1.0;
+}
+
 __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs a) {
   griddep_launch_dependents();
   griddep_wait();
@@ -619,9 +792,7 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
   const DevSlab s = a.slabs[k];
   const MatScalars sc = a.scal[k];
   const double rows = d.rows, cols = d.cols;
-  double scale = 1.0;
-  if (a.scale_rule == MUON_SCALE_MOONLIGHT) scale = (double)a.scale_k * sqrt(fmax(rows, cols));
-  else if (a.scale_rule == MUON_SCALE_KELLER) scale = sqrt(fmax(1.0, rows / cols));
+  const double scale = step_scale(a, d);
 
   double wdo = sc.wo, doo = sc.o2;  // <W, D O>, ||D O||^2
   int axis = 0;
@@ -642,7 +813,7 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
     cf.axis = 3;
     cf.pad = 0;
     a.coef[k] = cf;
-    if (a.stats != nullptr) {
+    if (a.stats != nullptr && !a.w_free) {
       const float nan = __int_as_float(0x7fc00000);
       muon_stats_t st;
       st.w_norm = static_cast<float>(sqrt(sc.w2));
@@ -710,7 +881,7 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
   cf.axis = axis;
   cf.pad = 0;
   a.coef[k] = cf;
-  if (a.stats != nullptr) {
+  if (a.stats != nullptr && !a.w_free) {  // else post_stats, after post_apply
     double ot2 = oo;
     if (a.mode == MUON_MODE_MUONGS && sc.w2 > 0.0) ot2 = oo - wdo * wdo / sc.w2;
     muon_stats_t st;
@@ -728,11 +899,25 @@ __global__ void __launch_bounds__(kThreads) post_finalize_kernel(const ElemArgs 
 // Same walk as the plain reduction: per 64-column band, two 32-row sub-tiles at a time
 // with all loads issued before the arithmetic and, for tall matrices, one shared-memory
 // transpose of the two slab tiles.
+// The statistics' sums of Muon and the two-sided mode, per block: ||W_t||^2,
+// <W_t, D O_raw> and ||D O_raw||^2 (post_stats applies the scale).
+__device__ __forceinline__ void apply_stats_flush(const ElemArgs& a, int k, float sw2, float swo,
+                                                  float so2, double (*red)[kThreads / 32]) {
+  double acc[3] = {sw2, swo, so2};
+  block_sum<3>(acc, red);
+  if (threadIdx.x == 0) {
+    atomicAdd(&a.asum[k].w2, acc[0]);
+    atomicAdd(&a.asum[k].wo, acc[1]);
+    atomicAdd(&a.asum[k].o2, acc[2]);
+  }
+}
+
 template <bool XF32>
 __global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs a) {
   griddep_launch_dependents();
   griddep_wait();
   __shared__ float tile[kRedGroup][kTC][kTR + 1];
+  __shared__ double red[3][kThreads / 32];
   const int b = blockIdx.x;
   const int k = find_matrix(a, b);
   const DevMat d = a.mats[k];
@@ -745,6 +930,8 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs 
   const bool vec = (d.flags & MAT_VEC_OK) != 0;
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
   const bool ns_only = a.ns_only != 0;
+  const bool st = a.apply_stats != 0;  // block-uniform
+  float sw2 = 0.f, swo = 0.f, so2 = 0.f;
   const float xs = slab_scale(a, k);
   MatCoef cf;
   cf.cw = cf.co = 0.f;
@@ -813,12 +1000,19 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_kernel(const ElemArgs 
         for (int e = 0; e < 8; ++e) {
           float f = xs * rowf;
           if ((cf.axis & 2) && e < valid[q]) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+          if (st && e < valid[q]) {
+            const float ot = f * o[q][e];  // D O_raw
+            sw2 = fmaf(w[q][e], w[q][e], sw2);
+            swo = fmaf(w[q][e], ot, swo);
+            so2 = fmaf(ot, ot, so2);
+          }
           w[q][e] = fmaf(cf.cw, w[q][e], cf.co * f * o[q][e]);
         }
         store8_f32(d.W + (int64_t)r * d.ld_w + c, vec, valid[q], w[q]);
       }
     }
   }
+  if (st) apply_stats_flush(a, k, sw2, swo, so2, red);
 }
 
 // post_apply with the W and slab loads staged in shared memory (cp.async, the ring of
@@ -827,6 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
   griddep_launch_dependents();
   griddep_wait();
   extern __shared__ uint8_t dsm_raw[];
+  __shared__ double red[3][kThreads / 32];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 127) &
                                              ~static_cast<uintptr_t>(127));
   const int b = blockIdx.x;
@@ -841,6 +1036,8 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
   const MatCoef cf = a.coef[k];
   const float xs = slab_scale(a, k);  // 1/(||U||+eps) when the slab holds U (no iteration)
+  const bool st = a.apply_stats != 0;  // block-uniform
+  float sw2 = 0.f, swo = 0.f, so2 = 0.f;
   const int nbr = min(sub_r, (d.rows - R0 + kTR - 1) / kTR);
   const int nbc = min(sub_c, (d.cols - C0 + kTC - 1) / kTC);
   const int nsub = nbr * nbc;
@@ -891,6 +1088,12 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
       for (int e = 0; e < 8; ++e) {
         float f = xs * rowf;
         if ((cf.axis & 2) && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+        if (st && e < valid) {
+          const float ot = f * o[e];  // D O_raw
+          sw2 = fmaf(w[e], w[e], sw2);
+          swo = fmaf(w[e], ot, swo);
+          so2 = fmaf(ot, ot, so2);
+        }
         w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
       }
       store8_f32(d.W + static_cast<int64_t>(r) * d.ld_w + c, true, valid, w);
@@ -898,6 +1101,36 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
     __syncthreads();  // every thread is done with this stage before it is refilled
   }
   cp_async_wait<0>();
+  if (st) apply_stats_flush(a, k, sw2, swo, so2, red);
+}
+
+// ------------------------------------------------------------------ post_stats
+// Statistics of Muon and the two-sided mode from the sums post_apply accumulated:
+// ||W_t||, <W_t, O> and ||O~|| with O = s D O_raw (O~ = O: no projection in these
+// modes). The two-sided mode reports ||W_t|| only, as post_finalize does for it.
+__global__ void __launch_bounds__(kThreads) post_stats_kernel(const ElemArgs a) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int k = blockIdx.x * kThreads + threadIdx.x;
+  if (k >= a.n) return;
+  const DevMat d = a.mats[k];
+  const ApplySums sc = a.asum[k];
+  muon_stats_t st;
+  st.w_norm = static_cast<float>(sqrt(sc.w2));
+  st.reserved = 0;
+  if (a.mode == MUON_MODE_TWOSIDED) {
+    const float nan = __int_as_float(0x7fc00000);
+    st.w_dot_o = st.o_norm = st.update_rms = nan;
+    st.equil_axis = 3;
+  } else {
+    const double scale = step_scale(a, d);
+    const double oo = scale * scale * sc.o2;
+    st.w_dot_o = static_cast<float>(scale * sc.wo);
+    st.o_norm = static_cast<float>(sqrt(oo));
+    st.update_rms = static_cast<float>(sqrt(oo / (double(d.rows) * d.cols)));
+    st.equil_axis = a.coef[k].axis;
+  }
+  a.stats[d.orig] = st;
 }
 
 }  // namespace
@@ -1078,6 +1311,9 @@ cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s) {
 }
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s) {
   if (a.total_tiles <= 0) return cudaSuccess;
+  if (a.w_free)
+    return a.x_fp32 ? launch_pdl(post_reduce_o_kernel<true>, a.o_total_tiles, s, a)
+                    : launch_pdl(post_reduce_o_kernel<false>, a.o_total_tiles, s, a);
   if (a.staged && !a.x_fp32 && !a.equilibrate) return launch_staged_impl<post_reduce_staged_kernel>(a, s);
   if (a.equilibrate)
     return a.x_fp32 ? launch_pdl(post_reduce_eq_kernel<true>, a.total_tiles, s, a)
@@ -1094,6 +1330,10 @@ cudaError_t launch_post_apply(const ElemArgs& a, cudaStream_t s) {
   if (a.staged && !a.x_fp32 && !a.ns_only) return launch_staged_impl<post_apply_staged_kernel>(a, s);
   return a.x_fp32 ? launch_pdl(post_apply_kernel<true>, a.total_tiles, s, a)
                   : launch_pdl(post_apply_kernel<false>, a.total_tiles, s, a);
+}
+cudaError_t launch_post_stats(const ElemArgs& a, cudaStream_t s) {
+  if (a.n <= 0 || !a.apply_stats) return cudaSuccess;
+  return launch_pdl(post_stats_kernel, (a.n + kThreads - 1) / kThreads, s, a);
 }
 
 }  // namespace muon

@@ -8,6 +8,17 @@
 
 namespace muon {
 
+constexpr int kOTileR = 64;   // O-only reduction: slab rows per block
+constexpr int kOTileC = 256;  // O-only reduction: slab columns per tile of the walk
+
+// Sums post_apply accumulates for the statistics of Muon and the two-sided mode.
+struct ApplySums {
+  double w2;   // ||W_t||_F^2
+  double wo;   // <W_t, D O_raw>_F (D the equilibration scaling, identity when off)
+  double o2;   // ||D O_raw||_F^2
+  double pad;
+};
+
 // Arguments of the memory-bound kernels.
 struct ElemArgs {
   const DevMat* mats;
@@ -33,11 +44,20 @@ struct ElemArgs {
   int32_t sub_r, sub_c; // super-tile = sub_r x sub_c sub-tiles of 32 x 64 (1..4 each)
   int32_t staged;       // plain reduction through a shared-memory ring (aligned W rows, bf16 slab)
   int32_t staged_in;    // ingest through the ring (also bf16 G with rows of 16-byte multiples)
+  // Muon and two-sided modes: the update needs no W-dependent scalar, so the reduction
+  // reads the slab alone (post_reduce_o_kernel, bands of kOTileR slab rows walked in
+  // kOTileC-column tiles) and post_apply accumulates the statistics' W sums
+  int32_t w_free;
+  int32_t apply_stats;  // w_free and statistics requested
+  const int32_t* o_tile_prefix;  // n+1 entries: first O-only reduction band of each matrix
+  int32_t o_total_tiles;
+  ApplySums* asum;      // n entries, zeroed with the per-matrix scalars
 };
 
 cudaError_t launch_ingest(const ElemArgs& a, cudaStream_t s);
 cudaError_t launch_post_reduce(const ElemArgs& a, cudaStream_t s);
 cudaError_t launch_post_finalize(const ElemArgs& a, cudaStream_t s);
 cudaError_t launch_post_apply(const ElemArgs& a, cudaStream_t s);
+cudaError_t launch_post_stats(const ElemArgs& a, cudaStream_t s);
 
 }  // namespace muon

@@ -63,11 +63,13 @@ struct muon_plan_s {
   std::vector<DevMat> dev;         // plan order
   std::vector<int64_t> eq_off;     // plan order
   std::vector<int32_t> tile_prefix;
+  std::vector<int32_t> o_tile_prefix;  // O-only reduction tiles (slab frame)
   int64_t eq_total = 0;
   int sub_r = 4, sub_c = 4;  // elementwise super-tile in 32 x 64 sub-tiles
   bool staged = false;       // staged (shared-memory ring) post_reduce and post_apply
   bool staged_in = false;    // staged ingest
-  size_t off_scal = 0, off_coef = 0, off_desc = 0, off_slabs = 0, off_tiles = 0;
+  size_t off_scal = 0, off_coef = 0, off_desc = 0, off_slabs = 0, off_tiles = 0, off_otiles = 0;
+  size_t off_asum = 0;
   size_t off_eq_o2 = 0, off_eq_wo = 0, ws_bytes = 0;
   // cached per workspace pointer and device
   void* ws_cached = nullptr;
@@ -278,13 +280,21 @@ void build_plan(muon_plan_s* p) {
     const int64_t t = int64_t((p->dev[i].rows + tr - 1) / tr) * ((p->dev[i].cols + tc - 1) / tc);
     p->tile_prefix[i + 1] = static_cast<int32_t>(p->tile_prefix[i] + t);
   }
+  p->o_tile_prefix.assign(n + 1, 0);
+  for (int i = 0; i < n; ++i) {
+    // a block walks a band of kOTileR slab rows across the whole width
+    const int sm = std::min(p->dev[i].rows, p->dev[i].cols);
+    p->o_tile_prefix[i + 1] = p->o_tile_prefix[i] + (sm + kOTileR - 1) / kOTileR;
+  }
   // workspace layout
   size_t off = align_up(sizeof(WsHeader), kAlign);
   p->off_scal = off;   off = align_up(off + sizeof(MatScalars) * n, kAlign);
+  p->off_asum = off;   off = align_up(off + sizeof(ApplySums) * n, kAlign);
   p->off_coef = off;   off = align_up(off + sizeof(MatCoef) * n, kAlign);
   p->off_desc = off;   off = align_up(off + sizeof(DevMat) * n, kAlign);
   p->off_slabs = off;  off = align_up(off + sizeof(DevSlab) * n, kAlign);
   p->off_tiles = off;  off = align_up(off + sizeof(int32_t) * (n + 1), kAlign);
+  p->off_otiles = off; off = align_up(off + sizeof(int32_t) * (n + 1), kAlign);
   p->off_eq_o2 = off;  off = align_up(off + sizeof(float) * p->eq_total, kAlign);
   p->off_eq_wo = off;  off = align_up(off + sizeof(float) * p->eq_total, kAlign);
   off = align_up(off, kSlabAlign);
@@ -451,11 +461,12 @@ muon_status_t bind_workspace(muon_plan_s* p, void* ws, int dev, cudaStream_t str
     }
   }
   // one upload of [desc | slabs | tiles]
-  const size_t lo = p->off_desc, hi = p->off_tiles + sizeof(int32_t) * (n + 1);
+  const size_t lo = p->off_desc, hi = p->off_otiles + sizeof(int32_t) * (n + 1);
   std::vector<uint8_t> host(hi - lo, 0);
   std::memcpy(host.data() + (p->off_desc - lo), p->dev.data(), sizeof(DevMat) * n);
   std::memcpy(host.data() + (p->off_slabs - lo), slabs.data(), sizeof(DevSlab) * n);
   std::memcpy(host.data() + (p->off_tiles - lo), p->tile_prefix.data(), sizeof(int32_t) * (n + 1));
+  std::memcpy(host.data() + (p->off_otiles - lo), p->o_tile_prefix.data(), sizeof(int32_t) * (n + 1));
   if (cudaMemcpyAsync(base + lo, host.data(), host.size(), cudaMemcpyHostToDevice, stream) !=
       cudaSuccess)
     return MUON_ERR_CUDA;
@@ -494,10 +505,10 @@ void fill_class_args(const muon_plan_s* p, uint8_t* base, size_t c, int phase, i
 }
 
 enum ProfKind { PK_INGEST = 0, PK_GRAM, PK_POLY, PK_APPLY, PK_REDUCE, PK_FINALIZE, PK_POST,
-                PK_NS_FUSED, PK_COUNT };
+                PK_NS_FUSED, PK_STATS, PK_COUNT };
 const char* const kProfNames[PK_COUNT] = {"ingest", "ns_gram", "ns_poly", "ns_apply",
                                           "post_reduce", "post_finalize", "post_apply",
-                                          "ns_fused"};
+                                          "ns_fused", "post_stats"};
 constexpr size_t kMaxProfRecs = 1 << 16;
 
 cudaEvent_t prof_event(muon_plan_s* p) {
@@ -545,6 +556,12 @@ double class_phase_flops(const ClassInfo& ci, int phase) {
   return f * ci.count;
 }
 
+// Muon and the two-sided mode: no step scalar depends on W, so the reduction reads
+// the Newton-Schulz slab alone and post_apply gathers the statistics' W sums.
+bool w_free_mode(const muon_plan_s* p) {
+  return !p->ns_only && (p->hp.mode == MUON_MODE_MUON || p->hp.mode == MUON_MODE_TWOSIDED);
+}
+
 double elem_bytes(const muon_plan_s* p, int kind) {
   const int ex = p->x_fp32 ? 4 : 2;
   double total = 0;
@@ -552,7 +569,7 @@ double elem_bytes(const muon_plan_s* p, int kind) {
     const double e = double(d.rows) * d.cols;
     const int eg = (d.flags & MAT_G_BF16) ? 2 : 4;
     if (kind == PK_INGEST) total += e * (p->ns_only ? eg + ex : eg + 8 + ex);
-    else if (kind == PK_REDUCE) total += e * (4 + ex);
+    else if (kind == PK_REDUCE) total += e * (w_free_mode(p) ? ex : 4 + ex);
     else if (kind == PK_POST) total += e * (p->ns_only ? eg + ex : 8 + ex);
   }
   return total;
@@ -565,7 +582,9 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int n = p->n;
   const muon_hparams_t& hp = p->hp;
-  if (cudaMemsetAsync(base + p->off_scal, 0, sizeof(MatScalars) * n, stream) != cudaSuccess)
+  // the per-matrix scalars and the statistics' sums of post_apply (adjacent)
+  if (cudaMemsetAsync(base + p->off_scal, 0, p->off_asum - p->off_scal + sizeof(ApplySums) * n, stream) !=
+      cudaSuccess)
     return MUON_ERR_CUDA;
   if (p->eq_total > 0) {
     if (cudaMemsetAsync(base + p->off_eq_o2, 0, p->off_eq_wo - p->off_eq_o2 + sizeof(float) * p->eq_total,
@@ -600,6 +619,11 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
   ea.sub_c = p->sub_c;
   ea.staged = p->staged ? 1 : 0;
   ea.staged_in = p->staged_in ? 1 : 0;
+  ea.w_free = w_free_mode(p) ? 1 : 0;
+  ea.apply_stats = (ea.w_free && stats != nullptr) ? 1 : 0;
+  ea.o_tile_prefix = reinterpret_cast<const int32_t*>(base + p->off_otiles);
+  ea.o_total_tiles = p->o_tile_prefix[n];
+  ea.asum = reinterpret_cast<ApplySums*>(base + p->off_asum);
 
   {
     ProfScope ps(p, stream);
@@ -738,7 +762,9 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
   }
 
   if (!p->ns_only) {
-    const bool need_reduce = hp.mode != MUON_MODE_MUON || p->equilibrate || stats != nullptr;
+    // MuonGS and MuonH need <W,O> and ||W|| before the update; Muon and the two-sided
+    // mode need O sums only with equilibration (their statistics come from post_apply)
+    const bool need_reduce = ea.w_free ? p->equilibrate : true;
     if (need_reduce) {
       ProfScope ps(p, stream);
       if (launch_post_reduce(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
@@ -748,9 +774,16 @@ muon_status_t enqueue_step(muon_plan_s* p, void* ws, muon_stats_t* stats, int nu
     if (launch_post_finalize(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
     ps.done(PK_FINALIZE, 0.0, 0.0);
   }
-  ProfScope ps(p, stream);
-  if (launch_post_apply(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
-  ps.done(PK_POST, 0.0, elem_bytes(p, PK_POST));
+  {
+    ProfScope ps(p, stream);
+    if (launch_post_apply(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    ps.done(PK_POST, 0.0, elem_bytes(p, PK_POST));
+  }
+  if (ea.apply_stats) {
+    ProfScope ps(p, stream);
+    if (launch_post_stats(ea, stream) != cudaSuccess) return MUON_ERR_CUDA;
+    ps.done(PK_STATS, 0.0, 0.0);
+  }
   return MUON_OK;
 }
 

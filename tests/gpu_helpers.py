@@ -57,6 +57,20 @@ def run_steps(B, torch, W0s, grads_per_step, hp, g_dtype, use_plan=True):
     return out
 
 
+def check_muon_stats_against_own_update(W_prev_gpu, Wg, st, ohp):
+    """Muon mode has no projection, so the step applied O = ((1 - lr wd) W_t - W_{t+1}) / lr
+    (float64 from the GPU's own fp32 W_t and W_{t+1}: about 1e-6 relative). The
+    statistics <W_t, O> and ||O|| must describe that O; this pins the sums post_apply
+    gathers for them, the scale included, far tighter than the oracle comparison can."""
+    if ohp.mode != "muon":
+        return
+    O = ((1.0 - ohp.lr * ohp.weight_decay) * W_prev_gpu - Wg) / ohp.lr
+    on, wn = np.linalg.norm(O), np.linalg.norm(W_prev_gpu)
+    assert abs(st["o_norm"] - on) <= 1e-4 * on + 1e-9, (st["o_norm"], on)
+    wo = float(np.sum(W_prev_gpu * O))
+    assert abs(st["w_dot_o"] - wo) <= 1e-4 * wn * on + 1e-9, (st["w_dot_o"], wo, wn * on)
+
+
 def compare_runs(gpu, W0s, grads_per_step, ohp, tol, check_stats=True):
     """Per matrix and per step: relative error of W_t, M_t and dW_t against the oracle."""
     worst = {"W": 0.0, "M": 0.0, "dW": 0.0}
@@ -76,6 +90,7 @@ def compare_runs(gpu, W0s, grads_per_step, ohp, tol, check_stats=True):
                 assert abs(st["w_norm"] - wn) <= 1e-5 * wn + 1e-12
                 assert abs(st["o_norm"] - r.o_norm) <= 2 * tol * r.o_norm + 1e-6
                 assert abs(st["update_rms"] - r.update_rms) <= 2 * tol * r.update_rms + 1e-6
+                check_muon_stats_against_own_update(W_prev_gpu, Wg, st, ohp)
             W_prev_gpu, W_prev_orc = Wg, r.W
     return worst
 
@@ -121,6 +136,7 @@ def check_step(W, M, G, Wg, Mg, W_prev_gpu, st, ohp, tol, worst):
     assert abs(st["w_norm"] - wn) <= 1e-5 * wn + 1e-12
     assert abs(st["o_norm"] - r.o_norm) <= 2 * tol * r.o_norm + 1e-6
     assert abs(st["update_rms"] - r.update_rms) <= 2 * tol * r.update_rms + 1e-6
+    check_muon_stats_against_own_update(W_prev_gpu, Wg, st, ohp)
     for k, e in (("W", eW), ("M", eM), ("dW", edW)):
         worst[k] = max(worst.get(k, 0.0), e)
     return r.W, r.M

@@ -167,6 +167,26 @@ def test_fp32_step_mixed_shapes_one_shot_api(env):
     H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs", wd=0.05), H.TOL_FP32)
 
 
+@pytest.mark.parametrize("eq", [False, True])
+def test_fp32_muon_step_statistics_from_post_apply(env, eq):
+    """Muon on the fp32 Newton-Schulz path: with equilibration the reduction reads the
+    fp32 slab alone (its row and column sums in the slab's frame, tall matrices
+    included); without it no reduction runs and every statistic comes from post_apply.
+    4 steps against the oracle at the fp32 tolerance."""
+    B, torch = env
+    shapes = [(5, 9), (64, 48), (100, 300), (300, 100), (257, 255)]
+    W0 = [H.seeded(r, c, 70 + i, 0.02) for i, (r, c) in enumerate(shapes)]
+    grads = [[H.seeded(r, c, 80 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
+             for t in range(4)]
+    hp = H.gpu_hp(B, mode="muon", wd=0.1, ns_fp32=True, equilibrate=eq)
+    gpu = H.run_steps(B, torch, W0, grads, hp, torch.float32)
+    ohp = H.oracle_hp(mode="muon", wd=0.1, equilibrate=eq)
+    if eq:
+        H.compare_runs_equilibrated(gpu, W0, grads, ohp, H.TOL_FP32)
+    else:
+        H.compare_runs(gpu, W0, grads, ohp, H.TOL_FP32)
+
+
 def test_muongs_invariants_on_gpu(env):
     """<W_t, O~> = 0 and ||W_{t+1}||^2 = ||W_t||^2 + lr^2 ||O~||^2 (wd = 0), at fp32 level."""
     B, torch = env
@@ -224,6 +244,9 @@ def test_two_sided_mode_ten_steps(env):
     H.compare_runs(gpu, W0, grads, ohp, H.TOL_FP32, check_stats=False)
     for t in range(10):
         assert all(st["equil_axis"] == 3 for st in gpu[t][2])
+        for i in range(len(shapes)):   # ||W_t|| of the GPU's own W_t (gathered by post_apply)
+            wn = np.linalg.norm(W0[i].astype(np.float64) if t == 0 else gpu[t - 1][0][i])
+            assert abs(gpu[t][2][i]["w_norm"] - wn) <= 1e-5 * wn
 
 
 def test_strided_unaligned_views_ten_steps(env):
@@ -428,26 +451,31 @@ def test_single_cta_variable_width_tiles_ragged_m(env, m):
     H.compare_runs(gpu, W0, grads, H.oracle_hp(mode="muongs"), H.TOL_BF16)
 
 
-@pytest.mark.parametrize("cols_tail,ns_steps,eq", [(8, 5, False), (4, 5, False), (3, 5, False),
-                                                   (8, 0, False), (8, 5, True), (8, 0, True)])
-def test_large_ragged_step_staged_kernels(env, cols_tail, ns_steps, eq):
-    """A step above 4M elements with MuonGS (which needs <W,O>, ||W||^2 and ||O||^2).
-    Every width a multiple of 8 (cols_tail 8): ingest, the reduction and post_apply all
-    stage their loads in shared memory; a width that is a multiple of 4 only (cols_tail 4,
-    bf16 gradient rows not 16-byte multiples): ingest keeps its register-staged kernel; an
-    odd width (cols_tail 3): all three do. With equilibration the reduction also takes
-    the per-row and per-column sums; with no Newton-Schulz iteration the slab holds U
-    and every kernel applies 1/(||U||+eps) itself. The sub-tiles end ragged in rows and
-    columns, include a tall (transposed) matrix, and two matrices smaller than one 32 x 64
-    sub-tile. 2 steps against the oracle."""
+@pytest.mark.parametrize("mode,cols_tail,ns_steps,eq", [
+    ("muongs", 8, 5, False), ("muongs", 4, 5, False), ("muongs", 3, 5, False),
+    ("muongs", 8, 0, False), ("muongs", 8, 5, True), ("muongs", 8, 0, True),
+    ("muon", 8, 5, False), ("muon", 8, 5, True), ("muon", 3, 5, True), ("muon", 8, 0, True)])
+def test_large_ragged_step_staged_kernels(env, mode, cols_tail, ns_steps, eq):
+    """A step above 4M elements. MuonGS needs <W,O>, ||W||^2 and ||O||^2 before the
+    update; Muon needs no sum of W, so its reduction reads the slab alone (only with
+    equilibration: ||O||^2 and the O^2 row / column sums, in the slab's frame) and
+    post_apply gathers the statistics' sums of W. Every width a multiple of 8
+    (cols_tail 8): ingest, the reduction and post_apply all stage their loads in shared
+    memory; a width that is a multiple of 4 only (cols_tail 4, bf16 gradient rows not
+    16-byte multiples): ingest keeps its register-staged kernel; an odd width
+    (cols_tail 3): all three do. With equilibration the reduction also takes the per-row
+    and per-column sums; with no Newton-Schulz iteration the slab holds U and every kernel
+    applies 1/(||U||+eps) itself. The tiles end ragged in rows and columns, include a
+    tall (transposed) matrix, and two matrices smaller than one 32 x 64 sub-tile. 2 steps
+    against the oracle."""
     B, torch = env
     shapes = [(1000, 2048 + cols_tail), (2056, 1000), (516, 1288), (17, 24), (40, 8)]
     W0 = [H.seeded(r, c, 2300 + i, 0.02) for i, (r, c) in enumerate(shapes)]
     grads = [[H.seeded_bf16(r, c, 2400 + 10 * t + i, 1e-3) for i, (r, c) in enumerate(shapes)]
              for t in range(2)]
-    hp = H.gpu_hp(B, mode="muongs", wd=0.1, ns_steps=ns_steps, equilibrate=eq)
+    hp = H.gpu_hp(B, mode=mode, wd=0.1, ns_steps=ns_steps, equilibrate=eq)
     gpu = H.run_steps(B, torch, W0, grads, hp, torch.bfloat16)
-    ohp = H.oracle_hp(mode="muongs", wd=0.1, ns_steps=ns_steps, equilibrate=eq)
+    ohp = H.oracle_hp(mode=mode, wd=0.1, ns_steps=ns_steps, equilibrate=eq)
     if eq:
         H.compare_runs_equilibrated(gpu, W0, grads, ohp, H.TOL_BF16)
     else:

@@ -1083,18 +1083,36 @@ __global__ void __launch_bounds__(kThreads, 4) post_apply_staged_kernel(const El
                      *reinterpret_cast<const uint16_t*>(st + kStgW + o_tall_off(lc + e) + lr * 2))
                  << 16);
       }
-      const float rowf = (cf.axis & 1) ? a.eq_o2[s.eq_off + r] : 1.f;
+      const float fr = xs * ((cf.axis & 1) ? a.eq_o2[s.eq_off + r] : 1.f);
+      if (cf.axis & 2) {  // block-uniform: a factor per column
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float f = xs * rowf;
-        if ((cf.axis & 2) && e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
-        if (st && e < valid) {
-          const float ot = f * o[e];  // D O_raw
-          sw2 = fmaf(w[e], w[e], sw2);
-          swo = fmaf(w[e], ot, swo);
-          so2 = fmaf(ot, ot, so2);
+        for (int e = 0; e < 8; ++e) {
+          float f = fr;
+          if (e < valid) f *= a.eq_o2[s.eq_off + d.rows + c + e];
+          if (st && e < valid) {
+            const float ot = f * o[e];  // D O_raw
+            sw2 = fmaf(w[e], w[e], sw2);
+            swo = fmaf(w[e], ot, swo);
+            so2 = fmaf(ot, ot, so2);
+          }
+          w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
         }
-        w[e] = fmaf(cf.cw, w[e], cf.co * f * o[e]);
+      } else {  // one factor for the thread's 8 elements
+        if (st) {
+          float two = 0.f, too = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            if (e < valid) {
+              sw2 = fmaf(w[e], w[e], sw2);
+              two = fmaf(w[e], o[e], two);
+              too = fmaf(o[e], o[e], too);
+            }
+          swo = fmaf(fr, two, swo);
+          so2 = fmaf(fr * fr, too, so2);
+        }
+        const float cof = cf.co * fr;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w[e] = fmaf(cf.cw, w[e], cof * o[e]);
       }
       store8_f32(d.W + static_cast<int64_t>(r) * d.ld_w + c, true, valid, w);
     }

@@ -19,11 +19,14 @@
 // per thread, 128-bit accesses when aligned; the reductions and post_apply take two
 // 32-row sub-tiles at a time, all their loads issued before any arithmetic). The
 // super-tile of each block is found by binary search over a per-matrix tile prefix.
-// Without equilibration and with aligned rows, the reduction instead stages its loads in
-// shared memory with cp.async (post_reduce_staged_kernel).
+// With aligned rows, ingest, post_apply and (without equilibration) the W-and-O
+// reduction instead stage their loads in shared memory with cp.async (the *_staged
+// kernels). The slab-only reduction walks bands of 64 slab rows across the width
+// (its own prefix of bands).
 // Per-matrix sums use one atomic per block; the equilibration row / column sums are
 // reduced inside the block (shuffles, and shared memory across warps for columns) and
-// use one atomic per row and per column of the super-tile.
+// use one atomic per row and per column of the super-tile (of the band's tile, in the
+// slab-only reduction).
 #include <cuda_runtime.h>
 
 #include <atomic>

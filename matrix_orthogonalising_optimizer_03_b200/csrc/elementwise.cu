@@ -469,7 +469,8 @@ __global__ void __launch_bounds__(kThreads, 3) post_reduce_eq_kernel(const ElemA
 // read from the Newton-Schulz slab alone (2 bytes per element in bf16) in the slab's
 // own frame, where a slab row is a W row (wide) or a W column (tall: the slab holds
 // O^T), so nothing is transposed. A block takes a band of kOTileR slab rows across the
-// whole width, in kOTileC-column tiles: each warp 8 rows, each lane 8 consecutive
+// whole width (or, in a plan with too few bands to fill the GPU, one of `chunks` equal
+// pieces of it), in kOTileC-column tiles: each warp 8 rows, each lane 8 consecutive
 // columns of a tile (eight 16-byte loads, two each in fp32, issued before the
 // arithmetic). In bf16 4 blocks per SM (64 registers) keep loads in flight while a
 // block sums; two register buffers with the next tile's loads issued ahead (2 blocks
@@ -553,8 +554,14 @@ __global__ void __launch_bounds__(kThreads, XF32 ? 2 : 4) post_reduce_o_kernel(c
   const DevSlab s = a.slabs[k];
   const bool tall = (d.flags & MAT_TRANSPOSED) != 0;
   const int sm = tall ? d.cols : d.rows, sn = tall ? d.rows : d.cols;  // slab rows, cols
-  const int R0 = (b - a.o_tile_prefix[k]) * kOTileR;
+  // blocks of a matrix: bands x chunks (a band's column walk in `chunks` pieces)
+  const int bands = (sm + kOTileR - 1) / kOTileR;
+  const int chunks = (a.o_tile_prefix[k + 1] - a.o_tile_prefix[k]) / bands;
+  const int t = b - a.o_tile_prefix[k];
+  const int R0 = (t / chunks) * kOTileR;
   const int ntc = (sn + kOTileC - 1) / kOTileC;
+  const int per = (ntc + chunks - 1) / chunks;
+  const int j0 = (t % chunks) * per, j1 = min(ntc, j0 + per);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int rw = R0 + warp * 8;
   const float xs = slab_scale(a, k);
@@ -583,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, XF32 ? 2 : 4) post_reduce_o_kernel(c
   };
   {
     OTileRegs<XF32> A;
-    for (int j = 0; j < ntc; ++j) {
+    for (int j = j0; j < j1; ++j) {
       o_tile_load<XF32>(A, s.xf, s.ldx, rw, sm, j * kOTileC + lane * 8, sn);
       tile(A, j);
     }

@@ -10,6 +10,7 @@ namespace muon {
 
 constexpr int kOTileR = 64;   // O-only reduction: slab rows per block
 constexpr int kOTileC = 256;  // O-only reduction: slab columns per tile of the walk
+constexpr int kOMinBlocks = 1024;  // fewer bands than this: split each band's walk
 
 // Sums post_apply accumulates for the statistics of Muon and the two-sided mode.
 struct ApplySums {

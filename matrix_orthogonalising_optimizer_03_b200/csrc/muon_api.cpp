@@ -280,11 +280,19 @@ void build_plan(muon_plan_s* p) {
     const int64_t t = int64_t((p->dev[i].rows + tr - 1) / tr) * ((p->dev[i].cols + tc - 1) / tc);
     p->tile_prefix[i + 1] = static_cast<int32_t>(p->tile_prefix[i] + t);
   }
+  // slab-only reduction: a block walks a band of kOTileR slab rows across the whole
+  // width; a plan with fewer than kOMinBlocks bands cuts each band's walk into up to
+  // `split` pieces (one block each), so that a few large matrices still fill the GPU
+  int64_t bands_total = 0;
+  for (int i = 0; i < n; ++i)
+    bands_total += (std::min(p->dev[i].rows, p->dev[i].cols) + kOTileR - 1) / kOTileR;
+  const int64_t split =
+      (bands_total == 0 || bands_total >= kOMinBlocks) ? 1 : (kOMinBlocks + bands_total - 1) / bands_total;
   p->o_tile_prefix.assign(n + 1, 0);
   for (int i = 0; i < n; ++i) {
-    // a block walks a band of kOTileR slab rows across the whole width
-    const int sm = std::min(p->dev[i].rows, p->dev[i].cols);
-    p->o_tile_prefix[i + 1] = p->o_tile_prefix[i] + (sm + kOTileR - 1) / kOTileR;
+    const int sm = std::min(p->dev[i].rows, p->dev[i].cols), sn = std::max(p->dev[i].rows, p->dev[i].cols);
+    const int64_t chunks = std::min<int64_t>(split, (sn + kOTileC - 1) / kOTileC);
+    p->o_tile_prefix[i + 1] = static_cast<int32_t>(p->o_tile_prefix[i] + ((sm + kOTileR - 1) / kOTileR) * chunks);
   }
   // workspace layout
   size_t off = align_up(sizeof(WsHeader), kAlign);

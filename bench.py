@@ -627,7 +627,7 @@ def measure_sharded(B, w, run, args, dev, world: int, rank: int, peaks, peak_src
 PER_SET = [("gpt160m", 0), ("gpt400m", 0), ("gpt400m", 1), ("moe_1b", 0), ("single_128x256", 0),
            ("single_128x256", 1)]
 
-# The surveyed NEXT rows that run as kernels of their own, each timed like a shape set:
+# The follow-on features that run as kernels of their own, each timed like a shape set:
 # the MuonH retraction and the two-sided normalisation on the 400M shapes (MuonW is the
 # Muon + weight-decay run of the same set, and the ZeRO-1 step is the "sharded" record).
 NEXT_RUNS = [("gpt400m", "muonh", 0.0), ("gpt400m", "twosided", 0.0)]
